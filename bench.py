@@ -1,0 +1,430 @@
+#!/usr/bin/env python
+"""Throughput of the LLSA hot path (pool -> select -> sparse attention forward
+-> sparse index transpose -> sparse attention backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...   (the CPU oracle, timed the same way)
+
+One step is one pass of the whole path over one batch of seeded synthetic
+input already resident in device memory.  Every GPU runs its own copy of the
+workload (heads and batches are independent, so the path shards with no
+collective): per-GPU work is fixed as N grows, i.e. weak scaling.  Rank 0
+prints one JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from hierarchical_top_sparse_llsa_b200 import workloads  # noqa: E402
+
+METRIC = "LLSA fwd+bwd ms & tokens/s at N=65536, % BF16 tensor peak, selection GB/s"
+UNIT = "tokens/s"
+STAGES = ("pool", "select", "fwd", "transpose", "bwd")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+SMS = 148
+FP32_LANES_PER_SM = 128
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        p["source"] = "measured"
+        return p
+    p = dict(FALLBACK_PEAKS)
+    p["source"] = "fallback"
+    return p
+
+
+def algorithmic_work(w: workloads.Workload) -> dict:
+    """Algorithmic bytes and FLOPs of one pass of each stage (no re-reads,
+    no gathers counted).  es = bytes per element of Q/K/V/O/dO/dQ/dK/dV."""
+    es = 2 if w.dtype == "bf16" else 4
+    BH, N, D, K, L = w.B * w.H, w.N, w.D, w.topk, w.L
+    fine = BH * N * D * es
+    nl = [w.n_level(l) for l in range(L + 1)]
+    keff = w.k_eff()
+    pyr_qk = sum(BH * nl[l] * D * 4 for l in range(1, L + 1))
+    pyr_v = sum(BH * nl[l] * D * 4 for l in range(2, L + 1))
+    idx_bytes = sum(BH * nl[l] * K * 4 for l in range(1, L + 1))
+    pairs = BH * N * w.keys_per_query()
+    cand = [0] * (L + 1)
+    cand[L] = nl[L]
+    for l in range(L - 1, 0, -1):
+        cand[l] = 16 * keff[l + 1]
+    work = {
+        "pool": {"bytes": 3 * fine + 2 * pyr_qk + pyr_v, "flops": 0, "bound": "hbm"},
+        # read Q(l), K(l) and the parent rows, write I(l); fp32 multiply + add per candidate channel
+        "select": {"bytes": 2 * pyr_qk + 2 * idx_bytes,
+                   "flops": sum(2 * D * BH * nl[l] * cand[l] for l in range(1, L + 1)),
+                   "bound": "alu"},
+        "fwd": {"bytes": 4 * fine + BH * N * 4, "flops": 4 * D * pairs, "bound": "hbm"},
+        "transpose": {"bytes": idx_bytes + idx_bytes + sum(BH * (nl[l] + 1) * 4 for l in range(1, L + 1)),
+                      "flops": 0, "bound": "hbm"},
+        "bwd": {"bytes": 8 * fine + 2 * BH * N * 4, "flops": 10 * D * pairs, "bound": "hbm"},
+    }
+    return work
+
+
+def launches_per_step(L: int) -> dict:
+    """Kernels each entry point launches (matches the C library's dispatch)."""
+    return {"pool": 1 + max(0, L - 2), "select": L, "fwd": 1, "transpose": 1,
+            "bwd": 2 + max(0, L - 1)}
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                sm.append(float(f[0]))
+                smax = float(f[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[3:7]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": smax, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gpu_selector(torch, dev):
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        return vis.split(",")[dev] if vis else str(dev)
+
+
+# ------------------------------------------------------------- CPU oracle
+def oracle_sample(w, x_head):
+    """The oracle's whole path on one head (a bounded sample of the workload)."""
+    import oracle
+
+    L, K = w.L, w.topk
+    scale = oracle.default_scale(w.D)
+    t0 = time.perf_counter()
+    pq, pk, pv = oracle.pool(x_head["q"], L), oracle.pool(x_head["k"], L), oracle.pool(x_head["v"], L)
+    idx = oracle.select_all(pq, pk, L, K)
+    O, LSE = oracle.attn_fwd(x_head["q"], x_head["k"], x_head["v"], pk, pv, idx, L, scale)
+    if w.backward:
+        for l in range(1, L + 1):
+            oracle.index_transpose(idx[l], w.n_level(l))
+        oracle.attn_bwd(x_head["q"], x_head["k"], x_head["v"], pk, pv, O, LSE, x_head["do"], idx, L, scale)
+    return time.perf_counter() - t0
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def cpu_sample_inputs(w):
+    x = workloads.make_inputs(w, heads=[0], with_dout=w.backward)
+    return x
+
+
+def config_of(w, world):
+    return {"workload": f"{w.name}: {w.side}x{w.side} pixels, N={w.N}, B={w.B}, H={w.H}, D={w.D}, "
+                        f"L={w.L}, K={w.topk}, {'fwd+bwd' if w.backward else 'fwd only'}",
+            "B": w.B, "H": w.H, "N": w.N, "D": w.D, "L": w.L, "topk": w.topk,
+            "l2": "inputs larger than L2 (no flush needed)",
+            "parallelism": f"replicas x{world} (no collective)"}
+
+
+# --------------------------------------------------------- reference arm
+def run_reference(args, rank, world):
+    w = workloads.WORKLOADS[args.workload]
+    if rank != 0:
+        return
+    x = cpu_sample_inputs(w)
+    for _ in range(args.warmup):
+        oracle_sample(w, x)
+    times = [oracle_sample(w, x) for _ in range(args.steps)]
+    t = sum(times) / len(times)
+    value = w.B * w.N / w.H / t  # one head of B*N tokens out of H
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": config_of(w, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"whole path on head 0 of {w.H} (B*N/H tokens per step)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------- our arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import hierarchical_top_sparse_llsa_b200 as llsa
+
+    w = workloads.WORKLOADS[args.workload]
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    peaks = load_peaks()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        nh = min(4, w.H)
+        xc = workloads.make_inputs(w, heads=slice(0, nh), with_dout=w.backward)
+        t = oracle_sample(w, xc)
+        cpu = {"value": w.B * w.N * nh / w.H / t, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": f"oracle whole path on heads 0..{nh - 1} of {w.H} ({t:.1f} s)"}
+
+    x = workloads.make_inputs(w, with_dout=w.backward)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    t_in = {k: torch.from_numpy(v).to(dev, dtype=tdt) for k, v in x.items()}
+    host = {k: torch.from_numpy(v).to(dtype=tdt).pin_memory() for k, v in x.items()}
+    del x
+    desc = llsa.make_desc(w.B, w.H, w.N, w.D, w.L, w.topk, llsa.BF16 if w.dtype == "bf16" else llsa.F32)
+    bufs = llsa.LlsaBuffers(desc, dev, with_bwd=w.backward)
+    o = torch.empty_like(t_in["q"])
+    lse = torch.empty(w.B, w.H, w.N, dtype=torch.float32, device=dev)
+    grads = [torch.empty_like(o) for _ in range(3)] if w.backward else []
+    stream = torch.cuda.current_stream(dev)
+    sh = stream.cuda_stream
+    st = bufs.status.data_ptr()
+
+    def step(tin, ev=None):
+        q, k, v = tin["q"].data_ptr(), tin["k"].data_ptr(), tin["v"].data_ptr()
+        if ev is not None:
+            ev[0].record(stream)
+        llsa.llsa_pool(desc, q, k, v, bufs.pyramid, sh)
+        if ev is not None:
+            ev[1].record(stream)
+        llsa.llsa_select(desc, bufs.pyramid, bufs.indices, sh)
+        if ev is not None:
+            ev[2].record(stream)
+        llsa.llsa_attn_fwd(desc, q, k, v, bufs.pyramid, bufs.indices, o.data_ptr(), lse.data_ptr(), st, sh)
+        if ev is not None:
+            ev[3].record(stream)
+        if w.backward:
+            llsa.llsa_index_transpose(desc, bufs.indices, bufs.csr, st, sh)
+            if ev is not None:
+                ev[4].record(stream)
+            dq, dk, dv = grads
+            llsa.llsa_attn_bwd(desc, q, k, v, bufs.pyramid, o.data_ptr(), lse.data_ptr(),
+                               tin["do"].data_ptr(), bufs.indices, bufs.csr, dq.data_ptr(),
+                               dk.data_ptr(), dv.data_ptr(), bufs.ws.data_ptr(), bufs.ws_bytes, st, sh)
+            if ev is not None:
+                ev[5].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step(t_in)
+    torch.cuda.synchronize()
+    if int(bufs.status.item()) != 0:
+        raise RuntimeError(f"device status {int(bufs.status.item())} during warm-up")
+
+    nst = 6 if w.backward else 4
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(gpu_selector(torch, local_rank)) if rank == 0 else None
+    if sampler:
+        sampler.__enter__()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for s in range(args.steps):
+        step(t_in, evs[s])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    if sampler:
+        sampler.__exit__()
+    ms = t_start.elapsed_time(t_end) / args.steps
+    stage_ms = {}
+    names = STAGES if w.backward else STAGES[:3]
+    for i, name in enumerate(names):
+        stage_ms[name] = statistics.mean(e[i].elapsed_time(e[i + 1]) for e in evs)
+
+    # end to end: pinned host inputs -> device -> path -> results back to pinned host
+    e2e_steps = max(1, min(args.steps, 5))
+    h_out = {"o": torch.empty(o.shape, dtype=o.dtype).pin_memory(),
+             "lse": torch.empty(lse.shape, dtype=lse.dtype).pin_memory()}
+    if w.backward:
+        for n in ("dq", "dk", "dv"):
+            h_out[n] = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    d_out = {"o": o, "lse": lse}
+    if w.backward:
+        d_out.update(dq=grads[0], dk=grads[1], dv=grads[2])
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+    barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        for k_, t_ in host.items():
+            t_in[k_].copy_(t_, non_blocking=True)
+        step(t_in)
+        for k_, t_ in d_out.items():
+            h_out[k_].copy_(t_, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+
+    if world > 1:
+        tt = torch.tensor([ms, e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms, e2e_ms = float(tt[0]), float(tt[1])
+    if int(bufs.status.item()) != 0:
+        raise RuntimeError(f"device status {int(bufs.status.item())}")
+    if rank != 0:
+        return
+
+    tokens = w.B * w.N
+    work = algorithmic_work(w)
+    hbm = peaks["hbm_gbs"]
+    tens = peaks["bf16_tflops_sustained"]
+    alu_peak = SMS * FP32_LANES_PER_SM * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12  # TFLOP/s, one op per lane-cycle
+    stages = {}
+    for n, t_ms in stage_ms.items():
+        wk = work[n]
+        gbs = wk["bytes"] / (t_ms * 1e-3) / 1e9
+        tfl = wk["flops"] / (t_ms * 1e-3) / 1e12
+        stages[n] = {"ms": round(t_ms, 4), "GB/s": round(gbs, 1), "TFLOP/s": round(tfl, 2),
+                     "frac_hbm": round(gbs / hbm, 4), "frac_bf16_tensor": round(tfl / tens, 4)}
+        if wk["bound"] == "alu":
+            stages[n]["frac_fp32_alu"] = round(tfl / alu_peak, 4)
+    dom = max(stage_ms, key=stage_ms.get)
+    wk = work[dom]
+    if wk["bound"] == "alu":
+        achieved = wk["flops"] / (stage_ms[dom] * 1e-3) / 1e12
+        roof = {"bound": "alu", "achieved": achieved, "peak": alu_peak, "unit": "TFLOP/s"}
+    else:
+        achieved = wk["bytes"] / (stage_ms[dom] * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = f"llsa_{'attn_' if dom in ('fwd', 'bwd') else ''}{dom} ({launches_per_step(w.L)[dom]} launches)"
+    roof["peak_source"] = f"{peaks['source']} (MEASURED_PEAKS.json)" if peaks["source"] == "measured" else "fallback"
+    attn_ms = stage_ms["fwd"] + stage_ms.get("bwd", 0.0)
+    attn_flops = work["fwd"]["flops"] + (work["bwd"]["flops"] if w.backward else 0)
+    sel_ms = stage_ms["pool"] + stage_ms["select"]
+    nlaunch = sum(launches_per_step(w.L)[n] for n in names)
+    line = {
+        "metric": METRIC, "value": world * tokens / (ms * 1e-3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": config_of(w, world),
+        "stages": stages,
+        "fwd_bwd_ms": attn_ms,
+        "fwd_bwd_frac_bf16_tensor": attn_flops / (attn_ms * 1e-3) / 1e12 / tens,
+        "selection_GBps": (work["pool"]["bytes"] + work["select"]["bytes"]) / (sel_ms * 1e-3) / 1e9,
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": {"value": world * tokens / (e2e_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+        "gpu_launches": nlaunch * args.steps,
+        "clocks": sampler.summary() if sampler else None,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=workloads.HEADLINE, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        ap.error("--warmup must be at least 3")
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,259 @@
+// Host side of the C ABI declared in include/llsa.h: argument checks, the
+// backward workspace layout and kernel dispatch.  No allocation, no state.
+
+#include <math.h>
+#include <string.h>
+
+#include "llsa_internal.cuh"
+
+namespace llsa {
+cudaError_t launch_attn_fwd_simt(const AttnParams& p, int dtype, cudaStream_t s);
+cudaError_t launch_attn_bwd_simt(const AttnParams& p, int dtype, cudaStream_t s);
+
+cudaError_t launch_attn_fwd(const AttnParams& p, int dtype, cudaStream_t s) {
+  return launch_attn_fwd_simt(p, dtype, s);
+}
+cudaError_t launch_attn_bwd(const AttnParams& p, int dtype, cudaStream_t s) {
+  return launch_attn_bwd_simt(p, dtype, s);
+}
+}  // namespace llsa
+
+using namespace llsa;
+
+namespace {
+
+inline int check_desc(const llsa_desc* d) {
+  if (d == nullptr) return LLSA_ERR_INVALID_ARG;
+  if (d->B < 1 || d->H < 1 || d->N < kBlock || d->D < 1 || d->L < 1 || d->topk < 1)
+    return LLSA_ERR_INVALID_ARG;
+  if (d->flags != 0) return LLSA_ERR_INVALID_ARG;
+  if (d->dtype != LLSA_F32 && d->dtype != LLSA_BF16) return LLSA_ERR_INVALID_ARG;
+  if (d->D != 64 && d->D != 128) return LLSA_ERR_UNSUPPORTED;
+  if (d->L > kMaxL || d->topk > kMaxK) return LLSA_ERR_UNSUPPORTED;
+  const long long span = 1LL << (4 * d->L);
+  if (d->N % span != 0) return LLSA_ERR_INVALID_ARG;
+  if ((long long)d->B * d->H > 65535) return LLSA_ERR_UNSUPPORTED;  // grid.y
+  if ((long long)(d->N / kBlock) * d->topk > 0x7fffffffLL) return LLSA_ERR_UNSUPPORTED;
+  if (!(d->sm_scale >= 0.f) || isinf(d->sm_scale)) return LLSA_ERR_INVALID_ARG;
+  for (int l = 2; l <= d->L; ++l)
+    if (!(d->level_w[l] >= 0.f) || isinf(d->level_w[l])) return LLSA_ERR_INVALID_ARG;
+  return LLSA_OK;
+}
+
+inline int n_level(const llsa_desc* d, int l) { return d->N >> (4 * l); }
+
+inline float scale_of(const llsa_desc* d) {
+  return d->sm_scale > 0.f ? d->sm_scale : 1.0f / sqrtf((float)d->D);
+}
+
+struct WsLayout {
+  size_t delta = 0;
+  size_t part[kMaxL + 1] = {};
+  size_t coarse[kMaxL + 1] = {};
+  size_t total = 0;
+};
+
+inline WsLayout ws_layout(const llsa_desc* d) {
+  WsLayout w;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off += (bytes + 255) & ~(size_t)255;
+    return o;
+  };
+  const size_t BH = (size_t)d->B * d->H;
+  w.delta = take(BH * d->N * sizeof(float));
+  for (int l = 2; l <= d->L; ++l)
+    w.part[l] = take(BH * (size_t)(d->N >> 8) * d->topk * 2 * d->D * sizeof(float));
+  for (int l = 2; l <= d->L; ++l)
+    w.coarse[l] = take(BH * (size_t)n_level(d, l) * 2 * d->D * sizeof(float));
+  w.total = off;
+  return w;
+}
+
+inline int launch_status(cudaError_t e) { return e == cudaSuccess ? LLSA_OK : LLSA_ERR_LAUNCH; }
+
+void fill_attn_common(AttnParams& p, const llsa_desc* d, const void* q, const void* k,
+                      const void* v, const llsa_pyramid* pyr, const llsa_indices* idx) {
+  memset(&p, 0, sizeof(p));
+  p.q = q;
+  p.k = k;
+  p.v = v;
+  for (int l = 1; l <= d->L; ++l) p.idx[l] = idx->idx[l];
+  for (int l = 2; l <= d->L; ++l) {
+    p.pk[l] = pyr->k[l];
+    p.pv[l] = pyr->v[l];
+    const float w = d->level_w[l] > 0.f ? d->level_w[l] : 1.0f;
+    p.logw[l] = logf(w);
+  }
+  p.B = d->B;
+  p.H = d->H;
+  p.N = d->N;
+  p.D = d->D;
+  p.L = d->L;
+  p.K = d->topk;
+  p.scale = scale_of(d);
+}
+
+bool coarse_kv_present(const llsa_desc* d, const llsa_pyramid* pyr) {
+  for (int l = 2; l <= d->L; ++l)
+    if (pyr->k[l] == nullptr || pyr->v[l] == nullptr) return false;
+  return true;
+}
+
+bool indices_present(const llsa_desc* d, const llsa_indices* idx) {
+  for (int l = 1; l <= d->L; ++l)
+    if (idx->idx[l] == nullptr) return false;
+  return true;
+}
+
+}  // namespace
+
+extern "C" {
+
+int llsa_version(void) { return 100; }
+
+const char* llsa_status_string(int status) {
+  switch (status) {
+    case LLSA_OK: return "ok";
+    case LLSA_ERR_INVALID_ARG: return "invalid argument";
+    case LLSA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case LLSA_ERR_LAUNCH: return "kernel launch failed";
+    case LLSA_ERR_WORKSPACE: return "workspace too small";
+    default: return "unknown status";
+  }
+}
+
+int llsa_pool(const llsa_desc* desc, const void* q, const void* k, const void* v,
+              const llsa_pyramid* out, void* stream) {
+  int st = check_desc(desc);
+  if (st != LLSA_OK) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || out == nullptr) return LLSA_ERR_INVALID_ARG;
+  PoolParams p;
+  memset(&p, 0, sizeof(p));
+  p.x[0] = q;
+  p.x[1] = k;
+  p.x[2] = v;
+  for (int l = 1; l <= desc->L; ++l) {
+    if (out->q[l] == nullptr || out->k[l] == nullptr) return LLSA_ERR_INVALID_ARG;
+    if (l >= 2 && out->v[l] == nullptr) return LLSA_ERR_INVALID_ARG;
+    p.lvl[0][l] = out->q[l];
+    p.lvl[1][l] = out->k[l];
+    p.lvl[2][l] = (l >= 2) ? out->v[l] : nullptr;
+  }
+  p.BH = desc->B * desc->H;
+  p.N = desc->N;
+  p.D = desc->D;
+  p.L = desc->L;
+  return launch_status(launch_pool(p, desc->dtype, (cudaStream_t)stream));
+}
+
+int llsa_select(const llsa_desc* desc, const llsa_pyramid* pyr, const llsa_indices* out,
+                void* stream) {
+  int st = check_desc(desc);
+  if (st != LLSA_OK) return st;
+  if (pyr == nullptr || out == nullptr || !indices_present(desc, out)) return LLSA_ERR_INVALID_ARG;
+  for (int l = 1; l <= desc->L; ++l)
+    if (pyr->q[l] == nullptr || pyr->k[l] == nullptr) return LLSA_ERR_INVALID_ARG;
+  const int BH = desc->B * desc->H;
+  for (int l = desc->L; l >= 1; --l) {
+    SelectParams p;
+    p.ql = pyr->q[l];
+    p.kl = pyr->k[l];
+    p.parent = (l == desc->L) ? nullptr : out->idx[l + 1];
+    p.out = out->idx[l];
+    p.n = n_level(desc, l);
+    p.K = desc->topk;
+    st = launch_status(launch_select_level(p, BH, desc->D, (cudaStream_t)stream));
+    if (st != LLSA_OK) return st;
+  }
+  return LLSA_OK;
+}
+
+int llsa_attn_fwd(const llsa_desc* desc, const void* q, const void* k, const void* v,
+                  const llsa_pyramid* pyr, const llsa_indices* idx, void* o, float* lse,
+                  int32_t* dev_status, void* stream) {
+  int st = check_desc(desc);
+  if (st != LLSA_OK) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || lse == nullptr ||
+      idx == nullptr || pyr == nullptr)
+    return LLSA_ERR_INVALID_ARG;
+  if (!indices_present(desc, idx) || !coarse_kv_present(desc, pyr)) return LLSA_ERR_INVALID_ARG;
+  AttnParams p;
+  fill_attn_common(p, desc, q, k, v, pyr, idx);
+  p.out = o;
+  p.lse = lse;
+  p.status = dev_status;
+  return launch_status(launch_attn_fwd(p, desc->dtype, (cudaStream_t)stream));
+}
+
+int llsa_index_transpose(const llsa_desc* desc, const llsa_indices* idx, const llsa_csr* out,
+                         int32_t* dev_status, void* stream) {
+  int st = check_desc(desc);
+  if (st != LLSA_OK) return st;
+  if (idx == nullptr || out == nullptr || !indices_present(desc, idx)) return LLSA_ERR_INVALID_ARG;
+  TransposeParams p;
+  memset(&p, 0, sizeof(p));
+  p.BH = desc->B * desc->H;
+  p.K = desc->topk;
+  p.status = dev_status;
+  p.nlev = desc->L;
+  int cta = 0;
+  for (int l = 1; l <= desc->L; ++l) {
+    if (out->row_ptr[l] == nullptr || out->col[l] == nullptr) return LLSA_ERR_INVALID_ARG;
+    TransposeLevel& t = p.lv[l - 1];
+    t.idx = idx->idx[l];
+    t.row_ptr = out->row_ptr[l];
+    t.col = out->col[l];
+    t.n = n_level(desc, l);
+    t.ranges = (t.n + 255) / 256;
+    t.cta_begin = cta;
+    cta += p.BH * t.ranges;
+  }
+  return launch_status(launch_transpose(p, (cudaStream_t)stream));
+}
+
+size_t llsa_bwd_workspace_bytes(const llsa_desc* desc) {
+  if (check_desc(desc) != LLSA_OK) return 0;
+  return ws_layout(desc).total;
+}
+
+int llsa_attn_bwd(const llsa_desc* desc, const void* q, const void* k, const void* v,
+                  const llsa_pyramid* pyr, const void* o, const float* lse, const void* dout,
+                  const llsa_indices* idx, const llsa_csr* csr, void* dq, void* dk, void* dv,
+                  void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
+  int st = check_desc(desc);
+  if (st != LLSA_OK) return st;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || lse == nullptr ||
+      dout == nullptr || idx == nullptr || csr == nullptr || pyr == nullptr || dq == nullptr ||
+      dk == nullptr || dv == nullptr || ws == nullptr)
+    return LLSA_ERR_INVALID_ARG;
+  if (((uintptr_t)ws & 255) != 0) return LLSA_ERR_INVALID_ARG;
+  if (!indices_present(desc, idx) || !coarse_kv_present(desc, pyr)) return LLSA_ERR_INVALID_ARG;
+  for (int l = 1; l <= desc->L; ++l)
+    if (csr->row_ptr[l] == nullptr || csr->col[l] == nullptr) return LLSA_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(desc);
+  if (ws_bytes < w.total) return LLSA_ERR_WORKSPACE;
+  AttnParams p;
+  fill_attn_common(p, desc, q, k, v, pyr, idx);
+  p.o = o;
+  p.lse_in = lse;
+  p.dout = dout;
+  for (int l = 1; l <= desc->L; ++l) {
+    p.row_ptr[l] = csr->row_ptr[l];
+    p.col[l] = csr->col[l];
+  }
+  char* base = static_cast<char*>(ws);
+  p.delta = reinterpret_cast<float*>(base + w.delta);
+  for (int l = 2; l <= desc->L; ++l) {
+    p.part[l] = reinterpret_cast<float*>(base + w.part[l]);
+    p.coarse[l] = reinterpret_cast<float*>(base + w.coarse[l]);
+  }
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.status = dev_status;
+  return launch_status(launch_attn_bwd(p, desc->dtype, (cudaStream_t)stream));
+}
+
+}  // extern "C"

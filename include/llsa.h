@@ -1,0 +1,202 @@
+/*
+ * llsa.h - C ABI of the B200 (sm_100a) Log-linear Sparse Attention library.
+ *
+ * The method is "Trainable Log-linear Sparse Attention for Efficient Diffusion
+ * Transformers" (arXiv 2512.16615).  Each entry point below cites the section
+ * of the howistudyai explainer of that paper which defines its operation.
+ *
+ * Conventions for every call
+ * --------------------------
+ *  - Tokens: N fine tokens per (batch, head) in Z-order (Step 5: Index
+ *    Reordering for Images), so 16 consecutive tokens are a 4x4 pixel tile.
+ *  - Levels: level 0 is the fine tokens; level l (1 <= l <= L) has
+ *    N_l = N / 16^l tokens, each the mean of 16 level-(l-1) tokens.  A level-1
+ *    token is a 16-token query/key block.  N must be a multiple of 16^L.
+ *  - Layout: every tensor is contiguous [B, H, tokens, D], D innermost.
+ *    Q, K, V, O, dO, dQ, dK, dV hold `dtype` elements; pyramids are fp32.
+ *  - Index lists I(l): int32 [B, H, N_l, topk].  Row q lists the level-l key
+ *    tokens kept for level-l query token q, ascending, padded with -1 at the
+ *    tail.  Kernels that read index lists use an entry iff it lies in
+ *    [0, N_l) and is larger than every entry used before it in the row; any
+ *    other entry is skipped and reported through `dev_status` (never a fault).
+ *  - Memory: the caller allocates and owns every buffer (device memory unless
+ *    stated otherwise).  The library allocates nothing and keeps no state
+ *    between calls.  Calls are asynchronous on `stream` (a cudaStream_t; NULL
+ *    is the legacy default stream); buffers must stay valid until the work on
+ *    the stream has finished.
+ *  - Host errors: the return value.  Arguments are checked before any launch;
+ *    on an error nothing is enqueued.
+ *  - Device errors: a bit set OR-ed into *dev_status (a device int32 the
+ *    caller zeroes and reads after synchronising), if dev_status is not NULL.
+ */
+#ifndef LLSA_H_
+#define LLSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define LLSA_API __attribute__((visibility("default")))
+#else
+#define LLSA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LLSA_MAX_LEVELS 6 /* L <= 6 */
+#define LLSA_MAX_TOPK 32  /* topk <= 32 */
+#define LLSA_BLOCK 16     /* tokens per block and pooling factor per level */
+
+/* element types of Q, K, V, O, dO, dQ, dK, dV */
+enum { LLSA_F32 = 0, LLSA_BF16 = 1 };
+
+/* host status (return values) */
+enum {
+  LLSA_OK = 0,
+  LLSA_ERR_INVALID_ARG = 1, /* NULL pointer, bad shape, N not a multiple of 16^L, ... */
+  LLSA_ERR_UNSUPPORTED = 2, /* D not in {64, 128}, topk > 32, L > 6, ... */
+  LLSA_ERR_LAUNCH = 3,      /* a kernel launch failed (cudaGetLastError) */
+  LLSA_ERR_WORKSPACE = 4    /* workspace smaller than llsa_bwd_workspace_bytes() */
+};
+
+/* device status bits (OR-ed into *dev_status) */
+enum {
+  LLSA_DEV_BAD_INDEX = 1,    /* an index entry outside [-1, N_l) was skipped */
+  LLSA_DEV_NONCANONICAL = 2, /* a duplicate, unsorted entry or a pad before a valid entry */
+  LLSA_DEV_TIMEOUT = 4       /* a bounded wait inside a kernel gave up */
+};
+
+/* Problem description (plain data, passed by pointer, read before launch). */
+typedef struct {
+  int B, H, N, D; /* batch, heads, fine tokens, head dim (64 or 128) */
+  int L;          /* number of pooled levels, 1 <= L <= LLSA_MAX_LEVELS */
+  int topk;       /* K, kept keys per level, 1 <= K <= LLSA_MAX_TOPK */
+  int dtype;      /* LLSA_F32 or LLSA_BF16 */
+  int flags;      /* reserved, must be 0 */
+  float sm_scale; /* softmax scale; 0 selects 1/sqrt(D) */
+  /* level_w[l], l = 2..L: weight of the coarse keys of level l (KV
+   * Reweighting; the paper's setting is 16^l).  0 selects 1.  Entries 0, 1 and
+   * above L are ignored. */
+  float level_w[LLSA_MAX_LEVELS + 1];
+} llsa_desc;
+
+/* fp32 pyramid, [B, H, N_l, D] per level; entry 0 is unused. */
+typedef struct {
+  float* q[LLSA_MAX_LEVELS + 1]; /* levels 1..L */
+  float* k[LLSA_MAX_LEVELS + 1]; /* levels 1..L */
+  float* v[LLSA_MAX_LEVELS + 1]; /* levels 2..L (level-1 pooled V is never a key) */
+} llsa_pyramid;
+
+/* I(l), int32 [B, H, N_l, topk] for l = 1..L; entry 0 is unused. */
+typedef struct {
+  int32_t* idx[LLSA_MAX_LEVELS + 1];
+} llsa_indices;
+
+/* Key-major lists per level l = 1..L: row_ptr int32 [B, H, N_l + 1] and
+ * col int32 [B, H, N_l * topk].  Row c of (b, h) is
+ * col[row_ptr[c] .. row_ptr[c+1]), the level-l query tokens that kept key c,
+ * ascending; offsets restart at 0 for every (b, h); col past row_ptr[N_l] is -1. */
+typedef struct {
+  int32_t* row_ptr[LLSA_MAX_LEVELS + 1];
+  int32_t* col[LLSA_MAX_LEVELS + 1];
+} llsa_csr;
+
+/*
+ * llsa_pool - hierarchical compression (Step 1; Building Blocks:
+ * Hierarchical Compression).
+ *   Q(l)[t] = mean of Q(l-1)[16t .. 16t+15] for l = 1..L, likewise K; V for
+ *   l = 2..L (V(1) is formed internally).  Sums run left to right in fp32 with
+ *   one rounding per addition and are then multiplied by 1/16, so the result
+ *   is reproducible bit for bit.
+ *   q, k, v: [B, H, N, D] of desc->dtype.  out: pyramid levels as listed in
+ *   llsa_pyramid (all required).
+ */
+LLSA_API int llsa_pool(const llsa_desc* desc, const void* q, const void* k, const void* v,
+              const llsa_pyramid* out, void* stream);
+
+/*
+ * llsa_select - hierarchical Top-K selection (Step 2; Building Blocks:
+ * Hierarchical Top-K Selection).
+ *   Level L: every level-L query token scores every level-L key token.
+ *   Level l < L: query token q scores only the 16 children of each key kept
+ *   by its parent q/16 in I(l+1).  Score = Q(l)[q] . K(l)[c], unscaled, in
+ *   fp32 summed over d = 0..D-1 left to right with one rounding per multiply
+ *   and per add (no FMA).  The min(K, #candidates) best scores are kept;
+ *   equal scores (IEEE ==) go to the lower key index.  Rows are stored
+ *   ascending with -1 padding.
+ *   pyr: q[l], k[l] for l = 1..L (from llsa_pool).  out: I(1..L), written.
+ */
+LLSA_API int llsa_select(const llsa_desc* desc, const llsa_pyramid* pyr, const llsa_indices* out,
+                void* stream);
+
+/*
+ * llsa_attn_fwd - sparse attention with hierarchical KV enrichment and KV
+ * reweighting (Step 3; Building Blocks: Hierarchical KV Enrichment, KV
+ * Reweighting).
+ *   For query i of block b (i / 16 == b) the keys are the 16 fine tokens of
+ *   every block in I(1)[b] (weight 1) and, for l = 2..L, the pooled tokens
+ *   K(l)[c], V(l)[c] for c in I(l)[b / 16^(l-1)] (weight level_w[l]):
+ *     s_ij = sm_scale * q_i . k_j
+ *     O_i  = sum_j w_j e^{s_ij} v_j / sum_j w_j e^{s_ij}
+ *     lse_i = ln sum_j w_j e^{s_ij}          (natural log)
+ *   A query without keys gets O_i = 0 and lse_i = -inf.
+ *   idx may be any caller-made index lists (no hierarchy consistency needed).
+ *   pyr: k[l], v[l] for l = 2..L.  o: [B, H, N, D] dtype.  lse: fp32 [B, H, N].
+ *   dev_status: may be NULL.
+ */
+LLSA_API int llsa_attn_fwd(const llsa_desc* desc, const void* q, const void* k, const void* v,
+                  const llsa_pyramid* pyr, const llsa_indices* idx, void* o, float* lse,
+                  int32_t* dev_status, void* stream);
+
+/*
+ * llsa_index_transpose - sparse index transpose (Step 4; Building Blocks:
+ * Sparse Index Transpose).
+ *   For each level l = 1..L and (b, h): count the query tokens that kept each
+ *   key token, prefix-sum the counts into row_ptr, and list the query tokens
+ *   of each key in ascending order in col.  No dense mask is formed; the
+ *   result is deterministic and uses no global atomics.
+ *   idx: I(1..L).  out: CSR of every level, written.  dev_status: may be NULL.
+ */
+LLSA_API int llsa_index_transpose(const llsa_desc* desc, const llsa_indices* idx, const llsa_csr* out,
+                         int32_t* dev_status, void* stream);
+
+/*
+ * llsa_bwd_workspace_bytes - device scratch size that llsa_attn_bwd needs
+ * for desc (0 on an invalid desc).
+ */
+LLSA_API size_t llsa_bwd_workspace_bytes(const llsa_desc* desc);
+
+/*
+ * llsa_attn_bwd - gradients of llsa_attn_fwd with the indices held fixed
+ * (Step 4: the key-major backward that the sparse index transpose serves).
+ *   With P_ij = w_j e^{s_ij - lse_i} and Delta_i = dO_i . O_i:
+ *     dS_ij = P_ij (dO_i . v_j - Delta_i)
+ *     dQ_i  = sm_scale * sum_j dS_ij k_j
+ *     dk_j  = sm_scale * sum_i dS_ij q_i ,  dv_j = sum_i P_ij dO_i
+ *   A fine key's gradient goes to its token; a level-l coarse key's gradient
+ *   is spread to each of its 16^l fine tokens divided by 16^l (the mean's
+ *   derivative).  Selection passes no gradient.  Sums run in a fixed order
+ *   without global atomics, so results are identical from run to run.
+ *   o, lse: the outputs of llsa_attn_fwd.  dout: dO.  csr: llsa_index_transpose
+ *   of the same idx.  dq, dk, dv: [B, H, N, D] dtype, written.
+ *   ws: device scratch of at least llsa_bwd_workspace_bytes(desc) bytes,
+ *   256-byte aligned.  dev_status: may be NULL.
+ */
+LLSA_API int llsa_attn_bwd(const llsa_desc* desc, const void* q, const void* k, const void* v,
+                  const llsa_pyramid* pyr, const void* o, const float* lse, const void* dout,
+                  const llsa_indices* idx, const llsa_csr* csr, void* dq, void* dk, void* dv,
+                  void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/* Static text for a host status code. */
+LLSA_API const char* llsa_status_string(int status);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+LLSA_API int llsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LLSA_H_ */

@@ -242,13 +242,13 @@ def attn_fwd(Q, K, V, pyr_k, pyr_v, idx, L, scale, level_w=None, block_chunk=512
                     {l: coarse[l][b, h, b0:b1] for l in coarse}, L, level_w)
                 q = np.asarray(Q[b, h, b0 * FACTOR:b1 * FACTOR], dtype=np.float64)
                 q = q.reshape(b1 - b0, FACTOR, D)
-                s = scale * np.einsum("bid,bjd->bij", q, ks) + lw[:, None, :]
+                s = scale * np.matmul(q, ks.transpose(0, 2, 1)) + lw[:, None, :]
                 s = np.where(ok[:, None, :], s, -np.inf)
                 m = s.max(axis=-1, keepdims=True)
                 has = np.isfinite(m)
                 e = np.where(ok[:, None, :], np.exp(s - np.where(has, m, 0.0)), 0.0)
                 den = e.sum(axis=-1, keepdims=True)
-                o = np.einsum("bij,bjd->bid", e, vs) / np.where(has, den, 1.0)
+                o = np.matmul(e, vs) / np.where(has, den, 1.0)
                 lse = np.where(has, m + np.log(np.where(has, den, 1.0)), -np.inf)
                 O[b, h, b0 * FACTOR:b1 * FACTOR] = o.reshape(-1, D)
                 LSE[b, h, b0 * FACTOR:b1 * FACTOR] = lse.reshape(-1)
@@ -328,15 +328,15 @@ def attn_bwd(Q, K, V, pyr_k, pyr_v, O, LSE, dO, idx, L, scale, level_w=None, blo
                 o = np.asarray(O[b, h, sl], dtype=np.float64).reshape(b1 - b0, FACTOR, D)
                 do = np.asarray(dO[b, h, sl], dtype=np.float64).reshape(b1 - b0, FACTOR, D)
                 lse = np.asarray(LSE[b, h, sl], dtype=np.float64).reshape(b1 - b0, FACTOR)
-                s = scale * np.einsum("bid,bjd->bij", q, ks) + lw[:, None, :]
+                s = scale * np.matmul(q, ks.transpose(0, 2, 1)) + lw[:, None, :]
                 fin = np.isfinite(lse)[..., None] & ok[:, None, :]
                 P = np.where(fin, np.exp(np.where(fin, s - lse[..., None], 0.0)), 0.0)
                 delta = (do * o).sum(axis=-1)  # [nb, 16]
-                dP = np.einsum("bid,bjd->bij", do, vs)
+                dP = np.matmul(do, vs.transpose(0, 2, 1))
                 dS = P * (dP - delta[..., None])
-                dQ[b, h, sl] = (scale * np.einsum("bij,bjd->bid", dS, ks)).reshape(-1, D)
-                dk = scale * np.einsum("bij,bid->bjd", dS, q)  # [nb, S, D]
-                dv = np.einsum("bij,bid->bjd", P, do)
+                dQ[b, h, sl] = (scale * np.matmul(dS, ks)).reshape(-1, D)
+                dk = scale * np.matmul(dS.transpose(0, 2, 1), q)  # [nb, S, D]
+                dv = np.matmul(P.transpose(0, 2, 1), do)
                 nf = fi.shape[-1]
                 m = fi >= 0
                 np.add.at(dK[b, h], fi[m], dk[:, :nf][m])

@@ -1,0 +1,128 @@
+"""Shared helpers of the tests: run the CUDA path through the C ABI on torch
+buffers, run the oracle on the same inputs, and compare."""
+
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+import hierarchical_top_sparse_llsa_b200 as llsa
+from hierarchical_top_sparse_llsa_b200 import workloads
+
+BF16_REL = 2e-2  # bf16 inputs: |a - b| <= 2e-2 * max(|b|, rms(b)) elementwise
+F32_ABS = 1e-4   # fp32 inputs: max-abs
+
+
+def clean_indices(I: np.ndarray, n: int):
+    """Apply the library's used-entry rule to index rows (entries used iff in
+    [0, n) and above the last used one); returns rows in the canonical
+    layout (ascending, -1 tail) and the status bits the kernels must report."""
+    I = np.asarray(I)
+    out = np.full(I.shape, -1, dtype=np.int32)
+    flags = 0
+    for pos in np.ndindex(*I.shape[:-1]):
+        last, seen_pad, kept = -1, False, []
+        for v in I[pos]:
+            v = int(v)
+            if v == -1:
+                seen_pad = True
+            elif v < -1 or v >= n:
+                flags |= llsa.DEV_BAD_INDEX
+            elif v <= last:
+                flags |= llsa.DEV_NONCANONICAL
+            else:
+                if seen_pad:
+                    flags |= llsa.DEV_NONCANONICAL
+                last = v
+                kept.append(v)
+        out[pos][: len(kept)] = kept
+    return out, flags
+
+
+def assert_close(got, want, dtype: str, what: str):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    assert got.shape == want.shape, (what, got.shape, want.shape)
+    fin = np.isfinite(want)
+    assert np.array_equal(np.isfinite(got), fin), f"{what}: non-finite pattern differs"
+    err = np.abs(got[fin] - want[fin])
+    if dtype == "f32":
+        worst = err.max(initial=0.0)
+        assert worst <= F32_ABS, f"{what}: max-abs {worst:.3g} > {F32_ABS}"
+    else:
+        rms = np.sqrt(np.mean(want[fin] ** 2)) if fin.any() else 0.0
+        bound = BF16_REL * np.maximum(np.abs(want[fin]), rms)
+        bad = err > bound
+        assert not bad.any(), (
+            f"{what}: {bad.sum()} of {bad.size} elements outside 2e-2*max(|ref|, rms); "
+            f"worst excess {np.max(err - bound):.3g}, max-abs {err.max():.3g}, rms {rms:.3g}")
+
+
+def run_gpu(B, H, N, D, L, topk, dtype, inputs, level_w=None, ext_idx=None, bwd=True,
+            device="cuda"):
+    """The whole path through the C ABI.  Returns numpy copies of everything."""
+    import torch
+
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    t = {k: torch.from_numpy(np.ascontiguousarray(v)).to(device=device, dtype=tdt) for k, v in inputs.items()}
+    desc = llsa.make_desc(B, H, N, D, L, topk, llsa.BF16 if dtype == "bf16" else llsa.F32,
+                          level_w=level_w)
+    bufs = llsa.LlsaBuffers(desc, device, with_bwd=bwd)
+    stream = torch.cuda.current_stream().cuda_stream
+    st = bufs.status.data_ptr()
+    llsa.llsa_pool(desc, t["q"].data_ptr(), t["k"].data_ptr(), t["v"].data_ptr(), bufs.pyramid, stream)
+    llsa.llsa_select(desc, bufs.pyramid, bufs.indices, stream)
+    torch.cuda.synchronize()
+    out = {"pq": {l: bufs.pq[l].cpu().numpy() for l in bufs.pq},
+           "pk": {l: bufs.pk[l].cpu().numpy() for l in bufs.pk},
+           "pv": {l: bufs.pv[l].cpu().numpy() for l in bufs.pv},
+           "sel": {l: bufs.idx[l].cpu().numpy() for l in bufs.idx}}
+    if ext_idx is not None:
+        for l, I in ext_idx.items():
+            bufs.idx[l].copy_(torch.from_numpy(np.ascontiguousarray(I, dtype=np.int32)))
+    o = torch.empty_like(t["q"])
+    lse = torch.empty(B, H, N, dtype=torch.float32, device=device)
+    llsa.llsa_attn_fwd(desc, t["q"].data_ptr(), t["k"].data_ptr(), t["v"].data_ptr(), bufs.pyramid,
+                       bufs.indices, o.data_ptr(), lse.data_ptr(), st, stream)
+    if bwd:
+        llsa.llsa_index_transpose(desc, bufs.indices, bufs.csr, st, stream)
+        dq, dk, dv = torch.empty_like(o), torch.empty_like(o), torch.empty_like(o)
+        llsa.llsa_attn_bwd(desc, t["q"].data_ptr(), t["k"].data_ptr(), t["v"].data_ptr(), bufs.pyramid,
+                           o.data_ptr(), lse.data_ptr(), t["do"].data_ptr(), bufs.indices, bufs.csr,
+                           dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), bufs.ws.data_ptr(),
+                           bufs.ws_bytes, st, stream)
+    torch.cuda.synchronize()
+    out["idx"] = {l: bufs.idx[l].cpu().numpy() for l in bufs.idx}
+    out["O"] = o.float().cpu().numpy()
+    out["LSE"] = lse.cpu().numpy()
+    if bwd:
+        out["row_ptr"] = {l: bufs.row_ptr[l].cpu().numpy() for l in bufs.row_ptr}
+        out["col"] = {l: bufs.col[l].cpu().numpy() for l in bufs.col}
+        out["dQ"] = dq.float().cpu().numpy()
+        out["dK"] = dk.float().cpu().numpy()
+        out["dV"] = dv.float().cpu().numpy()
+    out["status"] = int(bufs.status.item())
+    return out
+
+
+def run_oracle(inputs, L, topk, level_w=None, idx=None, bwd=True, pyr=None):
+    """The oracle on the same inputs.  ``idx`` replaces the selection;
+    ``pyr`` (a dict with pq, pk, pv) replaces the pooling."""
+    Q, K, V = inputs["q"], inputs["k"], inputs["v"]
+    D = Q.shape[-1]
+    scale = oracle.default_scale(D)
+    if pyr is None:
+        pyr = {"pq": oracle.pool(Q, L), "pk": oracle.pool(K, L), "pv": oracle.pool(V, L)}
+    sel = oracle.select_all(pyr["pq"], pyr["pk"], L, topk) if idx is None else idx
+    O, LSE = oracle.attn_fwd(Q, K, V, pyr["pk"], pyr["pv"], sel, L, scale, level_w)
+    res = {"pq": pyr["pq"], "pk": pyr["pk"], "pv": pyr["pv"], "idx": sel, "O": O, "LSE": LSE}
+    if bwd:
+        res["csr"] = {l: oracle.index_transpose(sel[l], Q.shape[2] // 16**l) for l in sel}
+        res["dQ"], res["dK"], res["dV"] = oracle.attn_bwd(
+            Q, K, V, pyr["pk"], pyr["pv"], O, LSE, inputs["do"], sel, L, scale, level_w)
+    return res
+
+
+def workload_inputs(name, heads=None):
+    w = workloads.WORKLOADS[name]
+    return w, workloads.make_inputs(w, heads=heads, with_dout=w.backward)

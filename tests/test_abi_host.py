@@ -1,0 +1,107 @@
+"""CPU-only checks of the C ABI: the library loads, exports every entry point
+that include/llsa.h declares, and its host-side argument checks reject bad
+calls before any launch (no GPU is touched: no call here reaches a kernel)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import hierarchical_top_sparse_llsa_b200 as llsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"LLSA_API\s+[\w\s\*]*?\b(llsa_\w+)\s*\(", text))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(llsa.LIB_PATH):
+        from hierarchical_top_sparse_llsa_b200 import build
+        build.build()
+    return llsa.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = _declared()
+    assert names == set(llsa.EXPORTED), names
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_status_strings(lib):
+    assert llsa.version() == 100
+    assert llsa.status_string(llsa.OK) == "ok"
+    assert "workspace" in llsa.status_string(llsa.ERR_WORKSPACE)
+
+
+def _desc(**kw):
+    base = dict(B=1, H=2, N=4096, D=64, L=3, topk=8, dtype=llsa.BF16)
+    base.update(kw)
+    return llsa.make_desc(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(D=96), llsa.ERR_UNSUPPORTED),
+    (dict(topk=33), llsa.ERR_UNSUPPORTED),
+    (dict(L=7, N=16**7), llsa.ERR_UNSUPPORTED),
+    (dict(N=4096 + 16), llsa.ERR_INVALID_ARG),  # not a multiple of 16^L
+    (dict(topk=0), llsa.ERR_INVALID_ARG),
+    (dict(dtype=5), llsa.ERR_INVALID_ARG),
+    (dict(B=0), llsa.ERR_INVALID_ARG),
+])
+def test_bad_descriptors_are_rejected_before_launch(lib, kw, status):
+    d = _desc(**kw)
+    pyr, ind, csr = llsa.LlsaPyramid(), llsa.LlsaIndices(), llsa.LlsaCsr()
+    fake = 256  # never dereferenced: the check fails first
+    assert llsa.llsa_pool(d, fake, fake, fake, pyr, check=False) == status
+    assert llsa.llsa_select(d, pyr, ind, check=False) == status
+    assert llsa.llsa_index_transpose(d, ind, csr, check=False) == status
+    assert llsa.llsa_bwd_workspace_bytes(d) == 0
+
+
+def test_null_buffers_are_rejected(lib):
+    d = _desc()
+    pyr, ind, csr = llsa.LlsaPyramid(), llsa.LlsaIndices(), llsa.LlsaCsr()
+    assert llsa.llsa_pool(d, None, None, None, pyr, check=False) == llsa.ERR_INVALID_ARG
+    assert llsa.llsa_pool(d, 256, 256, 256, pyr, check=False) == llsa.ERR_INVALID_ARG
+    assert llsa.llsa_select(d, pyr, ind, check=False) == llsa.ERR_INVALID_ARG
+    assert llsa.llsa_attn_fwd(d, 256, 256, 256, pyr, ind, 256, 256, check=False) == llsa.ERR_INVALID_ARG
+    assert llsa.llsa_index_transpose(d, ind, csr, check=False) == llsa.ERR_INVALID_ARG
+    with pytest.raises(llsa.LlsaError):
+        llsa.llsa_select(d, pyr, ind)
+
+
+def test_workspace_size_and_checks(lib):
+    d = _desc()
+    B, H, N, D, L, K = 1, 2, 4096, 64, 3, 8
+    r256 = lambda x: (x + 255) // 256 * 256
+    want = r256(B * H * N * 4)
+    want += sum(r256(B * H * (N // 256) * K * 2 * D * 4) for _ in range(2, L + 1))
+    want += sum(r256(B * H * (N // 16**l) * 2 * D * 4) for l in range(2, L + 1))
+    assert llsa.llsa_bwd_workspace_bytes(d) == want
+    # fill every pointer with a fake non-null value: the size check fails first
+    pyr, ind, csr = llsa.LlsaPyramid(), llsa.LlsaIndices(), llsa.LlsaCsr()
+    for l in range(1, L + 1):
+        pyr.q[l] = pyr.k[l] = pyr.v[l] = ind.idx[l] = csr.row_ptr[l] = csr.col[l] = 256
+    st = llsa.llsa_attn_bwd(d, 256, 256, 256, pyr, 256, 256, 256, ind, csr, 256, 256, 256,
+                            256, want - 1, check=False)
+    assert st == llsa.ERR_WORKSPACE
+    st = llsa.llsa_attn_bwd(d, 256, 256, 256, pyr, 256, 256, 256, ind, csr, 256, 256, 256,
+                            260, want, check=False)
+    assert st == llsa.ERR_INVALID_ARG  # workspace not 256-byte aligned
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(llsa, "LIB_PATH", str(tmp_path / "nope.so"))
+    monkeypatch.setattr(llsa, "_lib", None)
+    with pytest.raises(llsa.LlsaError):
+        llsa.lib()

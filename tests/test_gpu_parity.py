@@ -1,0 +1,162 @@
+"""GPU parity of the whole LLSA path (through the C ABI) against the oracle.
+
+Bar: pyramid, indices and key-major lists bit-exact; O, LSE, dQ, dK, dV within
+max-abs 1e-4 (fp32 inputs) or 2e-2 * max(|ref|, rms(ref)) per element (bf16
+inputs, against the fp64 oracle on the same bf16-rounded inputs).  Full-size
+workloads run whole on the GPU and are checked on sampled heads, for which the
+oracle runs on the head slice of the same draw (heads are independent).
+"""
+
+import numpy as np
+import pytest
+
+import hierarchical_top_sparse_llsa_b200 as llsa
+from hierarchical_top_sparse_llsa_b200 import workloads
+from llsa_testlib import assert_close, clean_indices, run_gpu, run_oracle
+
+pytestmark = pytest.mark.gpu
+
+
+def _compare(w, g, r, hs, bwd):
+    sl = (slice(None), hs)
+    for l in range(1, w.L + 1):
+        assert np.array_equal(g["pq"][l][sl], r["pq"][l]), f"Q pyramid level {l}"
+        assert np.array_equal(g["pk"][l][sl], r["pk"][l]), f"K pyramid level {l}"
+        if l >= 2:
+            assert np.array_equal(g["pv"][l][sl], r["pv"][l]), f"V pyramid level {l}"
+        assert np.array_equal(g["idx"][l][sl], r["idx"][l]), f"indices level {l}"
+    assert_close(g["O"][sl], r["O"], w.dtype, "O")
+    assert_close(g["LSE"][sl], r["LSE"], "f32" if w.dtype == "f32" else "bf16", "LSE")
+    if bwd:
+        for l in range(1, w.L + 1):
+            rp, col = r["csr"][l]
+            assert np.array_equal(g["row_ptr"][l][sl], rp), f"row_ptr level {l}"
+            assert np.array_equal(g["col"][l][sl], col), f"col level {l}"
+        for name in ("dQ", "dK", "dV"):
+            assert_close(g[name][sl], r[name], w.dtype, name)
+
+
+@pytest.mark.parametrize("name,heads", [
+    ("tiny_32x32_f32", None),
+    ("img64_bf16", None),
+    ("img128_bf16", [0, 11]),
+    ("img256_bf16", [0, 15]),
+])
+def test_workload_fwd_bwd(name, heads):
+    w = workloads.WORKLOADS[name]
+    x = workloads.make_inputs(w)
+    g = run_gpu(w.B, w.H, w.N, w.D, w.L, w.topk, w.dtype, x)
+    assert g["status"] == 0
+    hs = slice(None) if heads is None else heads
+    xs = x if heads is None else {k: np.ascontiguousarray(v[:, heads]) for k, v in x.items()}
+    r = run_oracle(xs, w.L, w.topk)
+    _compare(w, g, r, hs, True)
+
+
+@pytest.mark.parametrize("name", ["img512_k8_bf16", "img512_k32_bf16"])
+def test_workload_fwd_only_scaling(name):
+    w = workloads.WORKLOADS[name]
+    x = workloads.make_inputs(w, with_dout=False)
+    g = run_gpu(w.B, w.H, w.N, w.D, w.L, w.topk, w.dtype, x, bwd=False)
+    assert g["status"] == 0
+    heads = [5]
+    xs = {k: np.ascontiguousarray(v[:, heads]) for k, v in x.items()}
+    r = run_oracle(xs, w.L, w.topk, bwd=False)
+    _compare(w, g, r, heads, False)
+
+
+def _small(seed, B, H, N, D, dtype="bf16"):
+    rng = np.random.default_rng(seed)
+    x = {k: rng.standard_normal((B, H, N, D)).astype(np.float32) for k in ("q", "k", "v", "do")}
+    if dtype == "bf16":
+        x = {k: workloads.round_to_bf16(v) for k, v in x.items()}
+    return x
+
+
+def test_paper_level_weights():
+    w = workloads.WORKLOADS["img64_bf16"]
+    x = workloads.make_inputs(w)
+    lw = [0, 0] + [16.0**l for l in range(2, w.L + 1)]
+    g = run_gpu(w.B, w.H, w.N, w.D, w.L, w.topk, w.dtype, x, level_w=lw)
+    r = run_oracle(x, w.L, w.topk, level_w=lw)
+    _compare(w, g, r, slice(None), True)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_single_level_flat_topk(dtype):
+    # L = 1: every query block scores every block (the single-level baseline)
+    x = _small(21, 1, 3, 2048, 64, dtype)
+    g = run_gpu(1, 3, 2048, 64, 1, 8, dtype, x)
+    r = run_oracle(x, 1, 8)
+    w = workloads.Workload("flat", 1, 3, 2048, 64, dtype, 1, 8, 0)
+    _compare(w, g, r, slice(None), True)
+
+
+def test_topk_above_candidates_pads():
+    # K = 32 with one top-level token and 16 level-2 candidates: rows padded
+    x = _small(22, 1, 2, 4096, 64)
+    g = run_gpu(1, 2, 4096, 64, 3, 32, "bf16", x)
+    r = run_oracle(x, 3, 32)
+    w = workloads.Workload("k32", 1, 2, 4096, 64, "bf16", 3, 32, 0)
+    _compare(w, g, r, slice(None), True)
+    assert np.all(g["idx"][3][..., 1:] == -1) and np.all(g["idx"][2][..., 16:] == -1)
+
+
+def test_head_dim_128_backward():
+    x = _small(23, 2, 2, 4096, 128)
+    g = run_gpu(2, 2, 4096, 128, 2, 8, "bf16", x)
+    r = run_oracle(x, 2, 8)
+    w = workloads.Workload("d128", 2, 2, 4096, 128, "bf16", 2, 8, 0)
+    _compare(w, g, r, slice(None), True)
+
+
+def test_external_indices_garbage_is_skipped_and_reported():
+    B, H, N, D, L, K = 1, 2, 4096, 64, 3, 6
+    x = _small(24, B, H, N, D)
+    rng = np.random.default_rng(25)
+    ext = {}
+    for l in range(1, L + 1):
+        n = N // 16**l
+        I = rng.integers(-3, n + 3, size=(B, H, n, K)).astype(np.int32)
+        I[..., 0, :] = -1  # an empty row
+        ext[l] = I
+    ext[1][0, 0, 7] = [5, 5, 9, 2, -1, 11]  # duplicate, unsorted, pad before valid
+    clean = {}
+    want_flags = 0
+    for l in range(1, L + 1):
+        clean[l], f = clean_indices(ext[l], N // 16**l)
+        want_flags |= f
+    g = run_gpu(B, H, N, D, L, K, "bf16", x, ext_idx=ext)
+    r = run_oracle(x, L, K, idx=clean)
+    assert g["status"] == want_flags and want_flags == (llsa.DEV_BAD_INDEX | llsa.DEV_NONCANONICAL)
+    assert_close(g["O"], r["O"], "bf16", "O")
+    assert_close(g["LSE"], r["LSE"], "bf16", "LSE")
+    for l in range(1, L + 1):
+        rp, col = r["csr"][l]
+        assert np.array_equal(g["row_ptr"][l], rp) and np.array_equal(g["col"][l], col)
+    for name in ("dQ", "dK", "dV"):
+        assert_close(g[name], r[name], "bf16", name)
+
+
+def test_empty_key_sets_give_zero_output():
+    B, H, N, D, L, K = 1, 1, 1024, 64, 2, 4
+    x = _small(26, B, H, N, D)
+    ext = {1: np.full((B, H, 64, K), -1, np.int32), 2: np.full((B, H, 4, K), -1, np.int32)}
+    ext[1][0, 0, 10:] = [0, 1, 2, 3]
+    ext[2][0, 0, 1:] = [0, 1, 2, 3]
+    g = run_gpu(B, H, N, D, L, K, "bf16", x, ext_idx=ext)
+    r = run_oracle(x, L, K, idx=ext)
+    assert g["status"] == 0
+    assert np.all(g["O"][0, 0, :160] == 0) and np.all(np.isneginf(g["LSE"][0, 0, :160]))
+    assert_close(g["O"], r["O"], "bf16", "O")
+    for name in ("dQ", "dK", "dV"):
+        assert_close(g[name], r[name], "bf16", name)
+
+
+def test_runs_are_bitwise_deterministic():
+    w = workloads.WORKLOADS["img64_bf16"]
+    x = workloads.make_inputs(w)
+    a = run_gpu(w.B, w.H, w.N, w.D, w.L, w.topk, w.dtype, x)
+    b = run_gpu(w.B, w.H, w.N, w.D, w.L, w.topk, w.dtype, x)
+    for key in ("O", "LSE", "dQ", "dK", "dV"):
+        assert np.array_equal(a[key], b[key], equal_nan=True), key
