@@ -27,6 +27,7 @@ BLOCK = 16
 F32, BF16 = 0, 1
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_LAUNCH, ERR_WORKSPACE = 0, 1, 2, 3, 4
 DEV_BAD_INDEX, DEV_NONCANONICAL, DEV_TIMEOUT = 1, 2, 4
+NOALLOC_SCRATCH_BYTES = 16 << 20
 
 EXPORTED = (
     "llsa_pool",
@@ -35,6 +36,7 @@ EXPORTED = (
     "llsa_index_transpose",
     "llsa_bwd_workspace_bytes",
     "llsa_attn_bwd",
+    "llsa_attn_bwd_noalloc",
     "llsa_status_string",
     "llsa_version",
 )
@@ -89,6 +91,8 @@ def lib() -> ctypes.CDLL:
             "llsa_attn_bwd": (ctypes.c_int, [P(LlsaDesc), vp, vp, vp, P(LlsaPyramid), vp, vp, vp,
                                              P(LlsaIndices), P(LlsaCsr), vp, vp, vp, vp, ctypes.c_size_t,
                                              vp, vp]),
+            "llsa_attn_bwd_noalloc": (ctypes.c_int, [P(LlsaDesc), vp, vp, vp, P(LlsaPyramid), vp, vp, vp,
+                                                     P(LlsaIndices), P(LlsaCsr), vp, vp, vp, vp, vp]),
             "llsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
             "llsa_version": (ctypes.c_int, []),
         }
@@ -153,6 +157,17 @@ def llsa_attn_bwd(desc, q, k, v, pyramid, o, lse, dout, indices, csr, dq, dk, dv
     st = lib().llsa_attn_bwd(ctypes.byref(desc), q, k, v, ctypes.byref(pyramid), o, lse, dout,
                              ctypes.byref(indices), ctypes.byref(csr), dq, dk, dv, ws, ws_bytes,
                              dev_status, stream)
+    return _check(st) if check else st
+
+
+def llsa_attn_bwd_noalloc(desc, q, k, v, pyramid, o, lse, dout, indices, csr, dq, dk, dv,
+                          dev_status=None, stream=0, check=True):
+    """llsa_attn_bwd without a caller workspace: scratch comes from a fixed
+    16 MiB device array inside the library (for callers that cannot
+    allocate); problems needing more return ERR_WORKSPACE."""
+    st = lib().llsa_attn_bwd_noalloc(ctypes.byref(desc), q, k, v, ctypes.byref(pyramid), o, lse, dout,
+                                     ctypes.byref(indices), ctypes.byref(csr), dq, dk, dv, dev_status,
+                                     stream)
     return _check(st) if check else st
 
 

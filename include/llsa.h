@@ -189,6 +189,33 @@ LLSA_API int llsa_attn_bwd(const llsa_desc* desc, const void* q, const void* k, 
                   const llsa_indices* idx, const llsa_csr* csr, void* dq, void* dk, void* dv,
                   void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
 
+/*
+ * llsa_attn_bwd_noalloc - llsa_attn_bwd for callers that cannot allocate.
+ *   The paper has no counterpart: this is a convenience of this library.
+ *   Some callers cannot provide the backward's scratch buffer because they
+ *   cannot call cudaMalloc there (a plugin host without an allocator, a
+ *   runtime whose device memory is fixed at start-up, a latency-critical loop
+ *   where cudaMalloc may block).  This entry point takes the same arguments as
+ *   llsa_attn_bwd minus ws/ws_bytes and allocates nothing: its scratch is a
+ *   fixed device array of LLSA_NOALLOC_SCRATCH_BYTES inside the library, held
+ *   by every GPU that loads the library until the process exits.
+ *   - Sizes: if llsa_bwd_workspace_bytes(desc) exceeds
+ *     LLSA_NOALLOC_SCRATCH_BYTES the call returns LLSA_ERR_WORKSPACE and
+ *     enqueues nothing (use llsa_attn_bwd with your own workspace instead).
+ *   - Set-up: the first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture.
+ *   - Sharing: every call uses the same array, which keeps the last call's
+ *     contents (nothing in it needs to start at zero).  Calls whose work
+ *     overlaps on the GPU race on it and give wrong results: serialise them.
+ */
+#define LLSA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+LLSA_API int llsa_attn_bwd_noalloc(const llsa_desc* desc, const void* q, const void* k,
+                                   const void* v, const llsa_pyramid* pyr, const void* o,
+                                   const float* lse, const void* dout, const llsa_indices* idx,
+                                   const llsa_csr* csr, void* dq, void* dk, void* dv,
+                                   int32_t* dev_status, void* stream);
+
 /* Static text for a host status code. */
 LLSA_API const char* llsa_status_string(int status);
 
