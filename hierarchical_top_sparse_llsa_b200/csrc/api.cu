@@ -1,18 +1,19 @@
 // Host side of the C ABI declared in include/llsa.h: argument checks, the
 // backward workspace layout and kernel dispatch.  No allocation, no state.
 
+#include <cuda.h>
 #include <math.h>
 #include <string.h>
+
+#include <mutex>
 
 #include "llsa_internal.cuh"
 
 namespace llsa {
 cudaError_t launch_attn_fwd_simt(const AttnParams& p, int dtype, cudaStream_t s);
 cudaError_t launch_attn_bwd_simt(const AttnParams& p, int dtype, cudaStream_t s);
+cudaError_t launch_attn_fwd_mma(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s);
 
-cudaError_t launch_attn_fwd(const AttnParams& p, int dtype, cudaStream_t s) {
-  return launch_attn_fwd_simt(p, dtype, s);
-}
 cudaError_t launch_attn_bwd(const AttnParams& p, int dtype, cudaStream_t s) {
   return launch_attn_bwd_simt(p, dtype, s);
 }
@@ -72,6 +73,42 @@ inline WsLayout ws_layout(const llsa_desc* d) {
 }
 
 inline int launch_status(cudaError_t e) { return e == cudaSuccess ? LLSA_OK : LLSA_ERR_LAUNCH; }
+
+// cuTensorMapEncodeTiled, fetched from the driver once (no link-time libcuda).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// A bf16 [rows, D] row-major tensor seen by TMA as tiles of 16 rows x 64
+// columns (128 bytes) with 128-byte swizzle.
+int make_row_tile_map(CUtensorMap* map, const void* base, uint64_t rows, int D) {
+  EncodeTiledFn fn = encode_tiled();
+  if (fn == nullptr) return LLSA_ERR_LAUNCH;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) != 0) return LLSA_ERR_INVALID_ARG;
+  const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  const cuuint32_t box[2] = {64, 16};
+  const cuuint32_t estride[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? LLSA_OK : LLSA_ERR_LAUNCH;
+}
 
 void fill_attn_common(AttnParams& p, const llsa_desc* d, const void* q, const void* k,
                       const void* v, const llsa_pyramid* pyr, const llsa_indices* idx) {
@@ -184,7 +221,19 @@ int llsa_attn_fwd(const llsa_desc* desc, const void* q, const void* k, const voi
   p.out = o;
   p.lse = lse;
   p.status = dev_status;
-  return launch_status(launch_attn_fwd(p, desc->dtype, (cudaStream_t)stream));
+  if (desc->dtype == LLSA_F32)
+    return launch_status(launch_attn_fwd_simt(p, desc->dtype, (cudaStream_t)stream));
+  // bf16: tensor-core kernel with TMA gathers
+  if (((uintptr_t)o & 15) != 0) return LLSA_ERR_INVALID_ARG;
+  const uint64_t rows = (uint64_t)desc->B * desc->H * desc->N;
+  if (rows > 0x7fffffffULL) return LLSA_ERR_UNSUPPORTED;  // TMA row coordinates are int32
+  CUtensorMap maps[3];
+  const void* srcs[3] = {q, k, v};
+  for (int i = 0; i < 3; ++i) {
+    st = make_row_tile_map(&maps[i], srcs[i], rows, desc->D);
+    if (st != LLSA_OK) return st;
+  }
+  return launch_status(launch_attn_fwd_mma(p, maps, (cudaStream_t)stream));
 }
 
 int llsa_index_transpose(const llsa_desc* desc, const llsa_indices* idx, const llsa_csr* out,

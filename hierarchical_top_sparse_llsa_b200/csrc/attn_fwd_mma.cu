@@ -1,0 +1,345 @@
+// Sparse attention forward with hierarchical KV enrichment and KV
+// reweighting, bf16 tensor-core kernel (Step 3 of the howistudyai explainer
+// of "Trainable Log-linear Sparse Attention for Efficient Diffusion
+// Transformers").
+//
+// One warp owns one 16-token query block (the block is exactly the M = 16 of
+// the warp MMA).  Its selected 16-token key blocks are contiguous 16-row
+// tiles of K and V, gathered by 2D TMA loads (128-byte swizzle, no
+// multicast) into a 3-stage ring with one mbarrier per stage, so the next
+// tiles are in flight while the current one is multiplied.  A CTA holds 4
+// sibling query blocks (same level-2 ancestor), which share every coarse
+// key; the coarse K/V rows (fp32 pyramid) are converted once per CTA to bf16
+// tiles in shared memory, with ln(w_l) per key folded into the scores.
+// S = Q K^T and O += P V run on m16n8k16 bf16 MMAs with fp32 accumulation;
+// the softmax is online, in base 2, in fp32 registers.
+
+#include <math.h>
+
+#include "keyset.cuh"
+#include "sm100_ptx.cuh"
+
+namespace llsa {
+
+namespace {
+
+constexpr int kFwdWarps = 4;
+constexpr int kStages = 3;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct SoftmaxState {
+  float m[2];  // running max of rows g and g+8 (base-2 scaled scores)
+  float l[2];  // this thread's partial row sums
+};
+
+// Online-softmax update of a 16x16 score tile held in two m16n8 accumulators
+// (s[nt][0..1]: row g, keys 8nt+2t, 8nt+2t+1; s[nt][2..3]: row g+8), then
+// P (bf16 A fragment) and rescaling of the output accumulators.
+template <int NT>
+__device__ __forceinline__ void softmax_tile(float (&s)[2][4], const float (&lw)[2][2], float sc2,
+                                             SoftmaxState& st, float (&o)[NT][4],
+                                             uint32_t (&pa)[4]) {
+  float x[2][4];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    x[nt][0] = fmaf(s[nt][0], sc2, lw[nt][0]);
+    x[nt][1] = fmaf(s[nt][1], sc2, lw[nt][1]);
+    x[nt][2] = fmaf(s[nt][2], sc2, lw[nt][0]);
+    x[nt][3] = fmaf(s[nt][3], sc2, lw[nt][1]);
+  }
+  float mx0 = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
+  float mx1 = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
+  mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+  mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+  mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+  mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+  const float mn0 = fmaxf(st.m[0], mx0), mn1 = fmaxf(st.m[1], mx1);
+  // a row whose every score so far is -inf keeps corr = 1 and p = 0
+  const float c0 = (mn0 == -INFINITY) ? 1.f : exp2f(st.m[0] - mn0);
+  const float c1 = (mn1 == -INFINITY) ? 1.f : exp2f(st.m[1] - mn1);
+  const float b0 = (mn0 == -INFINITY) ? 0.f : mn0;
+  const float b1 = (mn1 == -INFINITY) ? 0.f : mn1;
+  float p[2][4];
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    p[nt][0] = exp2f(x[nt][0] - b0);
+    p[nt][1] = exp2f(x[nt][1] - b0);
+    p[nt][2] = exp2f(x[nt][2] - b1);
+    p[nt][3] = exp2f(x[nt][3] - b1);
+  }
+  st.l[0] = st.l[0] * c0 + (p[0][0] + p[0][1] + p[1][0] + p[1][1]);
+  st.l[1] = st.l[1] * c1 + (p[0][2] + p[0][3] + p[1][2] + p[1][3]);
+  st.m[0] = mn0;
+  st.m[1] = mn1;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    o[nt][0] *= c0;
+    o[nt][1] *= c0;
+    o[nt][2] *= c1;
+    o[nt][3] *= c1;
+  }
+  pa[0] = pack_bf16(p[0][0], p[0][1]);
+  pa[1] = pack_bf16(p[0][2], p[0][3]);
+  pa[2] = pack_bf16(p[1][0], p[1][1]);
+  pa[3] = pack_bf16(p[1][2], p[1][3]);
+}
+
+// S (16 x 16) = Q (16 x D, A fragments) . K_tile^T; the K tile is a swizzled
+// 16-row tile at `kt` (shared address).
+template <int D>
+__device__ __forceinline__ void qk_tile(const uint32_t (&qa)[D / 16][4], uint32_t kt, int lane,
+                                        float (&s)[2][4]) {
+  const int mi = lane >> 3;
+  const int krow = (mi >> 1) * 8 + (lane & 7);
+  const int kc = mi & 1;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    uint32_t b0, b1, b2, b3;
+    ldsm_x4(kt + swz(krow, 2 * kk + kc), b0, b1, b2, b3);
+    mma_bf16(s[0], qa[kk], b0, b1);
+    mma_bf16(s[1], qa[kk], b2, b3);
+  }
+}
+
+// O (16 x D) += P (16 x 16, A fragment) . V_tile (16 x D, swizzled at vt).
+template <int D>
+__device__ __forceinline__ void pv_tile(const uint32_t (&pa)[4], uint32_t vt, int lane,
+                                        float (&o)[D / 8][4]) {
+  const int mi = lane >> 3;
+  const int vrow = (mi & 1) * 8 + (lane & 7);
+  const int vc = mi >> 1;
+#pragma unroll
+  for (int nn = 0; nn < D / 16; ++nn) {
+    uint32_t b0, b1, b2, b3;
+    ldsm_x4_t(vt + swz(vrow, 2 * nn + vc), b0, b1, b2, b3);
+    mma_bf16(o[2 * nn], pa, b0, b1);
+    mma_bf16(o[2 * nn + 1], pa, b2, b3);
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kFwdWarps * 32)
+attn_fwd_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                    const __grid_constant__ CUtensorMap tv, AttnParams p, int nct) {
+  constexpr int TILE = 32 * D;  // bytes of a 16-row bf16 tile
+  constexpr int NT = D / 8;
+  constexpr int HALVES = D / 64;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int bh = blockIdx.y;
+  const int n1 = p.N >> 4;
+  const int b = blockIdx.x * kFwdWarps + warp;
+  const bool active = b < n1;
+  const int K = p.K;
+
+  unsigned char* wbase = sm + (size_t)warp * TILE * (1 + 2 * kStages);
+  unsigned char* ck = sm + (size_t)kFwdWarps * TILE * (1 + 2 * kStages);
+  unsigned char* cv = ck + (size_t)nct * TILE;
+  float* clw = reinterpret_cast<float*>(cv + (size_t)nct * TILE);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(clw + nct * 16);
+  int* clist = reinterpret_cast<int*>(bars + kFwdWarps * (kStages + 1));
+  __shared__ int s_nc;
+  __shared__ int flist_all[kFwdWarps][32];  // each warp's used fine blocks, ascending
+  int* flist = flist_all[warp];
+
+  const uint32_t qt = smem_u32(wbase);
+  const uint32_t bar0 = smem_u32(bars + warp * (kStages + 1));  // [0] = Q, [1..] = stages
+  auto stage_k = [&](int st) { return qt + (uint32_t)(1 + 2 * st) * TILE; };
+  auto stage_v = [&](int st) { return qt + (uint32_t)(2 + 2 * st) * TILE; };
+  auto bar_of = [&](int st) { return bar0 + 8u * (1 + st); };
+
+  int flags = 0;
+  // ---- this warp's fine blocks (lane s holds slot s of its row of I(1))
+  int my_blk = -1;
+  bool used = false;
+  if (active && lane < K) {
+    const int32_t* row = p.idx[1] + ((size_t)bh * n1 + b) * K;
+    used = row_entry_used(row, lane, n1, flags);
+    my_blk = row[lane];
+  }
+  const unsigned fmask = __ballot_sync(0xffffffffu, used);
+  const int nf = __popc(fmask);
+  if (used) flist[__popc(fmask & ((1u << lane) - 1u))] = my_blk;
+  __syncwarp();
+
+  // ---- coarse keys shared by the CTA (warp 0 builds the list)
+  if (warp == 0) {
+    int n = 0;
+    const int b0 = blockIdx.x * kFwdWarps;
+    for (int l = 2; l <= p.L; ++l) {
+      const int nl = p.N >> (4 * l);
+      const int a = b0 >> (4 * (l - 1));
+      bool u = false;
+      int c = -1;
+      if (lane < K) {
+        const int32_t* row = p.idx[l] + ((size_t)bh * nl + a) * K;
+        u = row_entry_used(row, lane, nl, flags);
+        c = row[lane];
+      }
+      const unsigned m = __ballot_sync(0xffffffffu, u);
+      if (u) clist[n + __popc(m & ((1u << lane) - 1u))] = (l << 24) | c;
+      n += __popc(m);
+    }
+    if (lane == 0) s_nc = n;
+  }
+  if (lane == 0) {
+    for (int i = 0; i <= kStages; ++i) mbar_init(bar0 + 8u * i, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const int nc = s_nc;
+  const int ncpad = (nc + 15) >> 4;
+  // coarse rows: fp32 pyramid -> bf16 swizzled tiles; padded keys are zero
+  // rows with weight -inf
+  for (int e = threadIdx.x; e < ncpad * 16 * (D / 8); e += blockDim.x) {
+    const int key = e / (D / 8), j = e % (D / 8);
+    uint4 kq = make_uint4(0, 0, 0, 0), vq = make_uint4(0, 0, 0, 0);
+    if (key < nc) {
+      const int l = clist[key] >> 24, c = clist[key] & 0xffffff;
+      const size_t off = ((size_t)bh * (p.N >> (4 * l)) + c) * D + 8 * j;
+      const float4* ks = reinterpret_cast<const float4*>(p.pk[l] + off);
+      const float4* vs = reinterpret_cast<const float4*>(p.pv[l] + off);
+      const float4 k0 = ks[0], k1 = ks[1], v0 = vs[0], v1 = vs[1];
+      kq = make_uint4(pack_bf16(k0.x, k0.y), pack_bf16(k0.z, k0.w), pack_bf16(k1.x, k1.y), pack_bf16(k1.z, k1.w));
+      vq = make_uint4(pack_bf16(v0.x, v0.y), pack_bf16(v0.z, v0.w), pack_bf16(v1.x, v1.y), pack_bf16(v1.z, v1.w));
+    }
+    const size_t dst = (size_t)(key >> 4) * TILE + swz(key & 15, j);
+    *reinterpret_cast<uint4*>(ck + dst) = kq;
+    *reinterpret_cast<uint4*>(cv + dst) = vq;
+  }
+  for (int e = threadIdx.x; e < ncpad * 16; e += blockDim.x)
+    clw[e] = (e < nc) ? p.logw[clist[e] >> 24] * kLog2e : -INFINITY;
+
+  // ---- issue Q and the first fine tiles
+  const size_t rowbase = (size_t)bh * p.N;
+  auto issue_block = [&](int r) {
+    if (lane == 0) {
+      const int blk = flist[r];
+      const int st = r % kStages;
+      mbar_arrive_expect_tx(bar_of(st), 2u * TILE);
+      const int y = (int)(rowbase + (size_t)blk * 16);
+#pragma unroll
+      for (int h = 0; h < HALVES; ++h) {
+        tma_load_2d(stage_k(st) + h * 2048, &tk, 64 * h, y, bar_of(st));
+        tma_load_2d(stage_v(st) + h * 2048, &tv, 64 * h, y, bar_of(st));
+      }
+    }
+  };
+  if (active) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar0, TILE);
+#pragma unroll
+      for (int h = 0; h < HALVES; ++h) tma_load_2d(qt + h * 2048, &tq, 64 * h, (int)(rowbase + (size_t)b * 16), bar0);
+    }
+    for (int r = 0; r < nf && r < kStages; ++r) issue_block(r);
+  }
+  __syncthreads();  // coarse tiles written
+  if (!active) return;
+
+  bool ok = mbar_wait_bounded(bar0, 0);
+  uint32_t qa[D / 16][4];
+  {
+    const int mi = lane >> 3;
+    const int row = (mi & 1) * 8 + (lane & 7);
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk)
+      ldsm_x4(qt + swz(row, 2 * kk + (mi >> 1)), qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
+  }
+  float o[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+  SoftmaxState st;
+  st.m[0] = st.m[1] = -INFINITY;
+  st.l[0] = st.l[1] = 0.f;
+  const float sc2 = p.scale * kLog2e;
+  const float zero_lw[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+
+  int r = 0;
+  for (; r < nf && ok; ++r) {
+    const int sidx = r % kStages;
+    ok = mbar_wait_bounded(bar_of(sidx), (uint32_t)((r / kStages) & 1));
+    if (!ok) break;
+    float s[2][4];
+    uint32_t pa[4];
+    qk_tile<D>(qa, stage_k(sidx), lane, s);
+    softmax_tile<NT>(s, zero_lw, sc2, st, o, pa);
+    pv_tile<D>(pa, stage_v(sidx), lane, o);
+    __syncwarp();
+    fence_proxy_async_smem();
+    if (r + kStages < nf) issue_block(r + kStages);
+  }
+  if (!ok) {
+    // give the copies already in flight a bounded chance to land, then stop
+    for (int q = r; q < nf && q < r + kStages; ++q)
+      mbar_wait_bounded(bar_of(q % kStages), (uint32_t)((q / kStages) & 1));
+    if (lane == 0) report_status(p.status, LLSA_DEV_TIMEOUT);
+    return;
+  }
+  for (int ct = 0; ct < ncpad; ++ct) {
+    float s[2][4];
+    uint32_t pa[4];
+    qk_tile<D>(qa, smem_u32(ck) + ct * TILE, lane, s);
+    float lw[2][2];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      lw[nt][0] = clw[ct * 16 + 8 * nt + 2 * t];
+      lw[nt][1] = clw[ct * 16 + 8 * nt + 2 * t + 1];
+    }
+    softmax_tile<NT>(s, lw, sc2, st, o, pa);
+    pv_tile<D>(pa, smem_u32(cv) + ct * TILE, lane, o);
+  }
+
+  // ---- epilogue: O = acc / l, LSE = ln(sum) = (m + log2 l) ln 2
+  float l0 = st.l[0], l1 = st.l[1];
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+  const float i0 = l0 > 0.f ? 1.f / l0 : 0.f;
+  const float i1 = l1 > 0.f ? 1.f / l1 : 0.f;
+  bf16* O = static_cast<bf16*>(p.out);
+  const size_t tok0 = rowbase + (size_t)b * 16 + g;
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    *reinterpret_cast<uint32_t*>(O + tok0 * D + 8 * nt + 2 * t) = pack_bf16(o[nt][0] * i0, o[nt][1] * i0);
+    *reinterpret_cast<uint32_t*>(O + (tok0 + 8) * D + 8 * nt + 2 * t) = pack_bf16(o[nt][2] * i1, o[nt][3] * i1);
+  }
+  if (t == 0) {
+    p.lse[tok0] = l0 > 0.f ? (st.m[0] + log2f(l0)) * kLn2 : -INFINITY;
+    p.lse[tok0 + 8] = l1 > 0.f ? (st.m[1] + log2f(l1)) * kLn2 : -INFINITY;
+  }
+  flags = __reduce_or_sync(0xffffffffu, flags);
+  if (lane == 0) report_status(p.status, flags);
+}
+
+template <int D>
+cudaError_t launch_typed(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s) {
+  constexpr int TILE = 32 * D;
+  const int nct = ((p.L - 1) * p.K + 15) / 16;
+  const size_t smem = 1024 + (size_t)kFwdWarps * TILE * (1 + 2 * kStages) + 2 * (size_t)nct * TILE +
+                      nct * 16 * sizeof(float) + kFwdWarps * (kStages + 1) * 8 + nct * 16 * sizeof(int);
+  cudaError_t e = cudaFuncSetAttribute(attn_fwd_mma_kernel<D>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int n1 = p.N / kBlock;
+  dim3 grid((n1 + kFwdWarps - 1) / kFwdWarps, p.B * p.H);
+  attn_fwd_mma_kernel<D><<<grid, kFwdWarps * 32, smem, s>>>(maps[0], maps[1], maps[2], p, nct);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// maps: Q, K, V as 2D [B*H*N rows, D cols] bf16, box 16 x 64, 128-byte swizzle.
+cudaError_t launch_attn_fwd_mma(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s) {
+  return (p.D == 64) ? launch_typed<64>(p, maps, s) : launch_typed<128>(p, maps, s);
+}
+
+}  // namespace llsa

@@ -153,7 +153,6 @@ struct AttnParams {
 cudaError_t launch_pool(const PoolParams& p, int dtype, cudaStream_t s);
 cudaError_t launch_select_level(const SelectParams& p, int BH, int D, cudaStream_t s);
 cudaError_t launch_transpose(const TransposeParams& p, cudaStream_t s);
-cudaError_t launch_attn_fwd(const AttnParams& p, int dtype, cudaStream_t s);
 cudaError_t launch_attn_bwd(const AttnParams& p, int dtype, cudaStream_t s);
 
 }  // namespace llsa
