@@ -13,10 +13,7 @@ namespace llsa {
 cudaError_t launch_attn_fwd_simt(const AttnParams& p, int dtype, cudaStream_t s);
 cudaError_t launch_attn_bwd_simt(const AttnParams& p, int dtype, cudaStream_t s);
 cudaError_t launch_attn_fwd_mma(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s);
-
-cudaError_t launch_attn_bwd(const AttnParams& p, int dtype, cudaStream_t s) {
-  return launch_attn_bwd_simt(p, dtype, s);
-}
+cudaError_t launch_attn_bwd_mma(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s);
 }  // namespace llsa
 
 using namespace llsa;
@@ -65,7 +62,7 @@ inline WsLayout ws_layout(const llsa_desc* d) {
   const size_t BH = (size_t)d->B * d->H;
   w.delta = take(BH * d->N * sizeof(float));
   for (int l = 2; l <= d->L; ++l)
-    w.part[l] = take(BH * (size_t)(d->N >> 8) * d->topk * 2 * d->D * sizeof(float));
+    w.part[l] = take(BH * (size_t)(d->N >> 7) * d->topk * 2 * d->D * sizeof(float));
   for (int l = 2; l <= d->L; ++l)
     w.coarse[l] = take(BH * (size_t)n_level(d, l) * 2 * d->D * sizeof(float));
   w.total = off;
@@ -302,7 +299,19 @@ int llsa_attn_bwd(const llsa_desc* desc, const void* q, const void* k, const voi
   p.dk = dk;
   p.dv = dv;
   p.status = dev_status;
-  return launch_status(launch_attn_bwd(p, desc->dtype, (cudaStream_t)stream));
+  if (desc->dtype == LLSA_F32)
+    return launch_status(launch_attn_bwd_simt(p, desc->dtype, (cudaStream_t)stream));
+  // bf16: tensor-core kernels with TMA gathers
+  if ((((uintptr_t)dq | (uintptr_t)dk | (uintptr_t)dv) & 15) != 0) return LLSA_ERR_INVALID_ARG;
+  const uint64_t rows = (uint64_t)desc->B * desc->H * desc->N;
+  if (rows > 0x7fffffffULL) return LLSA_ERR_UNSUPPORTED;  // TMA row coordinates are int32
+  CUtensorMap maps[4];
+  const void* srcs[4] = {q, k, v, dout};
+  for (int i = 0; i < 4; ++i) {
+    st = make_row_tile_map(&maps[i], srcs[i], rows, desc->D);
+    if (st != LLSA_OK) return st;
+  }
+  return launch_status(launch_attn_bwd_mma(p, maps, (cudaStream_t)stream));
 }
 
 }  // extern "C"

@@ -1,0 +1,571 @@
+// Backward of the enriched sparse attention, bf16 tensor-core kernels (the
+// key-major backward of Step 4 of the howistudyai explainer of "Trainable
+// Log-linear Sparse Attention for Efficient Diffusion Transformers";
+// Building Blocks: Sparse Index Transpose).
+//
+// Pass 1, query-major (bwd_q_mma_kernel): one warp per 16-token query block,
+// 8 sibling blocks per CTA (they share every coarse key).  Selected K/V tiles
+// arrive by 2D TMA loads into a 2-stage per-warp ring; the key list is
+// walked twice:
+//   sweep 1: S = Q K^T, dP = dO V^T, P = w e^{S - LSE}, Delta_i = sum_j P dP
+//            (from unrounded terms: O is stored rounded);
+//   sweep 2: dS = P (dP - Delta), dQ += dS K.
+// P and dS enter their MMAs as a bf16 hi + lo pair (about 16 mantissa bits):
+// the sums over queries in dK and dV cancel strongly on image-like inputs,
+// and single bf16 rounding of dS left some small dK entries 3x outside a
+// 2e-2 relative band.
+// Coarse keys then give dQ their share and, per CTA, the partials
+// sum_i dS_ij q_i and sum_i P_ij dO_i: each warp forms its block's part with
+// MMAs on register transposes (movmatrix), and the CTA adds the 8 parts in a
+// fixed warp order, so no atomics are used.
+//
+// Pass 3, key-major (bwd_kv_mma_kernel): one warp per 16-token key block walks
+// its row of the level-1 key-major lists (query blocks, ascending).  With the
+// key block as the MMA's M: S^T = K Q^T, dP^T = V dO^T, dV += P^T dO,
+// dK += dS^T Q.  The epilogue adds every coarse gradient divided by 16^l.
+// (Pass 2, the per-level coarse reduce, is shared with the fp32 path.)
+
+#include <math.h>
+
+#include "keyset.cuh"
+#include "mma_tiles.cuh"
+
+namespace llsa {
+
+namespace {
+
+constexpr int kQWarps = 8;   // query blocks per CTA in pass 1 (one partial group)
+constexpr int kKVWarps = 4;  // key blocks per CTA in pass 3
+constexpr int kRing = 2;
+constexpr float kLog2e = 1.4426950408889634f;
+
+__device__ __forceinline__ void zero_acc(float (&s)[2][4]) {
+#pragma unroll
+  for (int a = 0; a < 2; ++a)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[a][e] = 0.f;
+}
+
+// P = exp2(S * sc2 + lw - lse2) on a 16x16 tile (rows g, g+8 of the query
+// side); rows with lse = -inf get P = 0.
+__device__ __forceinline__ void probs_rows(const float (&s)[2][4], const float (&lw)[2][2], float sc2,
+                                           float lse_g, float lse_g8, float (&P)[2][4]) {
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float lse = (e < 2) ? lse_g : lse_g8;
+      const float x = fmaf(s[nt][e], sc2, lw[nt][e & 1] - lse);
+      P[nt][e] = (lse == -INFINITY) ? 0.f : exp2f(x);
+    }
+  }
+}
+
+__device__ __forceinline__ void pack_frag(const float (&x)[2][4], uint32_t (&a)[4]) {
+  a[0] = pack_bf16(x[0][0], x[0][1]);
+  a[1] = pack_bf16(x[0][2], x[0][3]);
+  a[2] = pack_bf16(x[1][0], x[1][1]);
+  a[3] = pack_bf16(x[1][2], x[1][3]);
+}
+
+// A fragment of the transpose of the 16x16 matrix whose A fragment is `a`.
+__device__ __forceinline__ void transpose_frag(const uint32_t (&a)[4], uint32_t (&t)[4]) {
+  t[0] = movmatrix_t(a[0]);
+  t[1] = movmatrix_t(a[2]);
+  t[2] = movmatrix_t(a[1]);
+  t[3] = movmatrix_t(a[3]);
+}
+
+// acc (16 x D) = A (16 x 16) . X (16 x D) where X's A fragments are `xa`
+// (X rows = the contraction index): the B fragments of X are the transposes
+// of its 8x8 sub-blocks.
+template <int D>
+__device__ __forceinline__ void mm_with_rowfrags(const uint32_t (&a)[4], const uint32_t (&xa)[D / 16][4],
+                                                 float (&acc)[D / 8][4]) {
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    mma_bf16(acc[2 * kk], a, movmatrix_t(xa[kk][0]), movmatrix_t(xa[kk][1]));
+    mma_bf16(acc[2 * kk + 1], a, movmatrix_t(xa[kk][2]), movmatrix_t(xa[kk][3]));
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kQWarps * 32)
+bwd_q_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                 const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
+                 AttnParams p, int nct) {
+  constexpr int TILE = 32 * D;
+  constexpr int NT = D / 8;
+  constexpr int HALVES = D / 64;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int bh = blockIdx.y;
+  const int grp = blockIdx.x;
+  const int n1 = p.N >> 4;
+  const int b = grp * kQWarps + warp;
+  const bool active = b < n1;
+  const int K = p.K;
+
+  unsigned char* wbase = sm + (size_t)warp * TILE * 2 * kRing;
+  unsigned char* ck = sm + (size_t)kQWarps * TILE * 2 * kRing;
+  unsigned char* cv = ck + (size_t)nct * TILE;
+  float* clw = reinterpret_cast<float*>(cv + (size_t)nct * TILE);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(clw + nct * 16);
+  int* clist = reinterpret_cast<int*>(bars + kQWarps * (1 + kRing));
+  int* cslot = clist + nct * 16;
+  __shared__ int s_nc;
+  __shared__ int flist_all[kQWarps][32];
+  int* flist = flist_all[warp];
+
+  const uint32_t w0 = smem_u32(wbase);
+  const uint32_t bar0 = smem_u32(bars + warp * (1 + kRing));
+  auto ring_k = [&](int st) { return w0 + (uint32_t)(2 * st) * TILE; };
+  auto ring_v = [&](int st) { return w0 + (uint32_t)(2 * st + 1) * TILE; };
+  auto bar_of = [&](int st) { return bar0 + 8u * (1 + st); };
+
+  int flags = 0;
+  int my_blk = -1;
+  bool used = false;
+  if (active && lane < K) {
+    const int32_t* row = p.idx[1] + ((size_t)bh * n1 + b) * K;
+    used = row_entry_used(row, lane, n1, flags);
+    my_blk = row[lane];
+  }
+  const unsigned fmask = __ballot_sync(0xffffffffu, used);
+  const int nf = __popc(fmask);
+  if (used) flist[__popc(fmask & ((1u << lane) - 1u))] = my_blk;
+  __syncwarp();
+
+  if (warp == 0) {
+    int n = 0;
+    const int b0 = grp * kQWarps;
+    for (int l = 2; l <= p.L; ++l) {
+      const int nl = p.N >> (4 * l);
+      const int a = b0 >> (4 * (l - 1));
+      bool u = false;
+      int c = -1;
+      if (lane < K) {
+        const int32_t* row = p.idx[l] + ((size_t)bh * nl + a) * K;
+        u = row_entry_used(row, lane, nl, flags);
+        c = row[lane];
+      }
+      const unsigned m = __ballot_sync(0xffffffffu, u);
+      if (u) {
+        const int pos = n + __popc(m & ((1u << lane) - 1u));
+        clist[pos] = (l << 24) | c;
+        cslot[pos] = lane;
+      }
+      n += __popc(m);
+    }
+    if (lane == 0) s_nc = n;
+  }
+  if (lane == 0) {
+    for (int i = 0; i <= kRing; ++i) mbar_init(bar0 + 8u * i, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const int nc = s_nc;
+  const int ncpad = (nc + 15) >> 4;
+  for (int e = threadIdx.x; e < ncpad * 16 * (D / 8); e += blockDim.x) {
+    const int key = e / (D / 8), j = e % (D / 8);
+    uint4 kq = make_uint4(0, 0, 0, 0), vq = make_uint4(0, 0, 0, 0);
+    if (key < nc) {
+      const int l = clist[key] >> 24, c = clist[key] & 0xffffff;
+      const size_t off = ((size_t)bh * (p.N >> (4 * l)) + c) * D + 8 * j;
+      const float4* ks = reinterpret_cast<const float4*>(p.pk[l] + off);
+      const float4* vs = reinterpret_cast<const float4*>(p.pv[l] + off);
+      const float4 k0 = ks[0], k1 = ks[1], v0 = vs[0], v1 = vs[1];
+      kq = make_uint4(pack_bf16(k0.x, k0.y), pack_bf16(k0.z, k0.w), pack_bf16(k1.x, k1.y), pack_bf16(k1.z, k1.w));
+      vq = make_uint4(pack_bf16(v0.x, v0.y), pack_bf16(v0.z, v0.w), pack_bf16(v1.x, v1.y), pack_bf16(v1.z, v1.w));
+    }
+    const size_t dst = (size_t)(key >> 4) * TILE + swz(key & 15, j);
+    *reinterpret_cast<uint4*>(ck + dst) = kq;
+    *reinterpret_cast<uint4*>(cv + dst) = vq;
+  }
+  for (int e = threadIdx.x; e < ncpad * 16; e += blockDim.x)
+    clw[e] = (e < nc) ? p.logw[clist[e] >> 24] * kLog2e : -INFINITY;
+
+  const size_t rowbase = (size_t)bh * p.N;
+  const int ntiles = 2 * nf;  // the fine key list is walked twice
+  auto issue = [&](int r) {
+    if (lane == 0) {
+      const int blk = flist[r % nf];
+      const int st = r % kRing;
+      mbar_arrive_expect_tx(bar_of(st), 2u * TILE);
+      const int y = (int)(rowbase + (size_t)blk * 16);
+#pragma unroll
+      for (int h = 0; h < HALVES; ++h) {
+        tma_load_2d(ring_k(st) + h * 2048, &tk, 64 * h, y, bar_of(st));
+        tma_load_2d(ring_v(st) + h * 2048, &tv, 64 * h, y, bar_of(st));
+      }
+    }
+  };
+  if (active && lane == 0) {
+    // Q and dO of this block land in the first ring stage before the ring starts
+    mbar_arrive_expect_tx(bar0, 2u * TILE);
+    const int y = (int)(rowbase + (size_t)b * 16);
+#pragma unroll
+    for (int h = 0; h < HALVES; ++h) {
+      tma_load_2d(ring_k(0) + h * 2048, &tq, 64 * h, y, bar0);
+      tma_load_2d(ring_v(0) + h * 2048, &tdo, 64 * h, y, bar0);
+    }
+  }
+  __syncthreads();  // coarse tiles written
+
+  bool ok = true;
+  uint32_t qa[D / 16][4], da[D / 16][4];
+  float lse_g = 0.f, lse_g8 = 0.f, delta_g = 0.f, delta_g8 = 0.f;
+  float dq[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) dq[nt][0] = dq[nt][1] = dq[nt][2] = dq[nt][3] = 0.f;
+  const float sc2 = p.scale * kLog2e;
+  const float zero_lw[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+  if (active) {
+    ok = mbar_wait_bounded(bar0, 0);
+    load_a_frags<D>(ring_k(0), lane, qa);
+    load_a_frags<D>(ring_v(0), lane, da);
+    const size_t tok0 = rowbase + (size_t)b * 16 + g;
+    lse_g = p.lse_in[tok0] * kLog2e;
+    lse_g8 = p.lse_in[tok0 + 8] * kLog2e;
+    __syncwarp();
+    fence_proxy_async_smem();
+    for (int r = 0; r < ntiles && r < kRing; ++r) issue(r);
+
+    // sweep 1: Delta
+    float dp0 = 0.f, dp1 = 0.f;
+    int r = 0;
+    for (; r < nf && ok; ++r) {
+      const int st = r % kRing;
+      ok = mbar_wait_bounded(bar_of(st), (uint32_t)((r / kRing) & 1));
+      if (!ok) break;
+      float s[2][4], dpv[2][4], P[2][4];
+      qk_tile<D>(qa, ring_k(st), lane, s);
+      qk_tile<D>(da, ring_v(st), lane, dpv);
+      probs_rows(s, zero_lw, sc2, lse_g, lse_g8, P);
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        dp0 += P[nt][0] * dpv[nt][0] + P[nt][1] * dpv[nt][1];
+        dp1 += P[nt][2] * dpv[nt][2] + P[nt][3] * dpv[nt][3];
+      }
+      __syncwarp();
+      fence_proxy_async_smem();
+      if (r + kRing < ntiles) issue(r + kRing);
+    }
+    for (int ct = 0; ct < ncpad && ok; ++ct) {
+      float s[2][4], dpv[2][4], P[2][4], lw[2][2];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        lw[nt][0] = clw[ct * 16 + 8 * nt + 2 * t];
+        lw[nt][1] = clw[ct * 16 + 8 * nt + 2 * t + 1];
+      }
+      qk_tile<D>(qa, smem_u32(ck) + ct * TILE, lane, s);
+      qk_tile<D>(da, smem_u32(cv) + ct * TILE, lane, dpv);
+      probs_rows(s, lw, sc2, lse_g, lse_g8, P);
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        dp0 += P[nt][0] * dpv[nt][0] + P[nt][1] * dpv[nt][1];
+        dp1 += P[nt][2] * dpv[nt][2] + P[nt][3] * dpv[nt][3];
+      }
+    }
+    dp0 += __shfl_xor_sync(0xffffffffu, dp0, 1);
+    dp0 += __shfl_xor_sync(0xffffffffu, dp0, 2);
+    dp1 += __shfl_xor_sync(0xffffffffu, dp1, 1);
+    dp1 += __shfl_xor_sync(0xffffffffu, dp1, 2);
+    delta_g = dp0;
+    delta_g8 = dp1;
+    if (t == 0) {
+      p.delta[tok0] = delta_g;
+      p.delta[tok0 + 8] = delta_g8;
+    }
+    // sweep 2: dQ from the fine keys
+    for (; r < ntiles && ok; ++r) {
+      const int st = r % kRing;
+      ok = mbar_wait_bounded(bar_of(st), (uint32_t)((r / kRing) & 1));
+      if (!ok) break;
+      float s[2][4], dpv[2][4], P[2][4];
+      qk_tile<D>(qa, ring_k(st), lane, s);
+      qk_tile<D>(da, ring_v(st), lane, dpv);
+      probs_rows(s, zero_lw, sc2, lse_g, lse_g8, P);
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) P[nt][e] *= dpv[nt][e] - ((e < 2) ? delta_g : delta_g8);
+      uint32_t dsh[4], dsl[4];
+      split_frag(P, dsh, dsl);
+      pv_tile2<D>(dsh, dsl, ring_k(st), lane, dq);
+      __syncwarp();
+      fence_proxy_async_smem();
+      if (r + kRing < ntiles) issue(r + kRing);
+    }
+    if (!ok) {
+      for (int q = r; q < ntiles && q < r + kRing; ++q)
+        mbar_wait_bounded(bar_of(q % kRing), (uint32_t)((q / kRing) & 1));
+      flags |= LLSA_DEV_TIMEOUT;
+    }
+  }
+
+  // coarse keys: dQ share and the per-CTA partials, reduced in warp order
+  const int NG = n1 / kQWarps;
+  float* stage = reinterpret_cast<float*>(wbase);  // [2][16][D] fp32, reuses this warp's ring
+  for (int ct = 0; ct < ncpad; ++ct) {
+    if (active && ok) {
+      float s[2][4], dpv[2][4], P[2][4], dS[2][4], lw[2][2];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        lw[nt][0] = clw[ct * 16 + 8 * nt + 2 * t];
+        lw[nt][1] = clw[ct * 16 + 8 * nt + 2 * t + 1];
+      }
+      qk_tile<D>(qa, smem_u32(ck) + ct * TILE, lane, s);
+      qk_tile<D>(da, smem_u32(cv) + ct * TILE, lane, dpv);
+      probs_rows(s, lw, sc2, lse_g, lse_g8, P);
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dS[nt][e] = P[nt][e] * (dpv[nt][e] - ((e < 2) ? delta_g : delta_g8));
+      uint32_t dsh[4], dsl[4], ph[4], pl[4], dsth[4], dstl[4], pth[4], ptl[4];
+      split_frag(dS, dsh, dsl);
+      split_frag(P, ph, pl);
+      pv_tile2<D>(dsh, dsl, smem_u32(ck) + ct * TILE, lane, dq);
+      transpose_frag(dsh, dsth);
+      transpose_frag(dsl, dstl);
+      transpose_frag(ph, pth);
+      transpose_frag(pl, ptl);
+      // part (16 coarse keys x D): rows g, g+8 of the transposed products
+      {
+        float acc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+        mm_with_rowfrags<D>(dsth, qa, acc);
+        mm_with_rowfrags<D>(dstl, qa, acc);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          *reinterpret_cast<float2*>(stage + g * D + 8 * nt + 2 * t) = make_float2(acc[nt][0], acc[nt][1]);
+          *reinterpret_cast<float2*>(stage + (g + 8) * D + 8 * nt + 2 * t) = make_float2(acc[nt][2], acc[nt][3]);
+        }
+      }
+      {
+        float acc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+        mm_with_rowfrags<D>(pth, da, acc);
+        mm_with_rowfrags<D>(ptl, da, acc);
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          *reinterpret_cast<float2*>(stage + 16 * D + g * D + 8 * nt + 2 * t) = make_float2(acc[nt][0], acc[nt][1]);
+          *reinterpret_cast<float2*>(stage + 16 * D + (g + 8) * D + 8 * nt + 2 * t) = make_float2(acc[nt][2], acc[nt][3]);
+        }
+      }
+    } else {
+      float* stg = stage;
+      for (int e = lane; e < 32 * D; e += 32) stg[e] = 0.f;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < 32 * D; e += blockDim.x) {
+      const int kv = e / (16 * D), key = (e / D) % 16, d = e % D;
+      const int ck_idx = ct * 16 + key;
+      if (ck_idx >= nc) continue;
+      float a = 0.f;
+      for (int w = 0; w < kQWarps; ++w)
+        a += reinterpret_cast<const float*>(sm + (size_t)w * TILE * 2 * kRing)[e];
+      const int l = clist[ck_idx] >> 24;
+      float* part = p.part[l] + ((((size_t)bh * NG + grp) * K + cslot[ck_idx]) * 2 + kv) * D + d;
+      *part = (kv == 0) ? a * p.scale : a;
+    }
+    __syncthreads();
+  }
+
+  if (active) {
+    bf16* dQ = static_cast<bf16*>(p.dq);
+    const size_t tok0 = rowbase + (size_t)b * 16 + g;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      *reinterpret_cast<uint32_t*>(dQ + tok0 * D + 8 * nt + 2 * t) =
+          pack_bf16(dq[nt][0] * p.scale, dq[nt][1] * p.scale);
+      *reinterpret_cast<uint32_t*>(dQ + (tok0 + 8) * D + 8 * nt + 2 * t) =
+          pack_bf16(dq[nt][2] * p.scale, dq[nt][3] * p.scale);
+    }
+  }
+  flags = __reduce_or_sync(0xffffffffu, flags);
+  if (lane == 0) report_status(p.status, flags);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kKVWarps * 32)
+bwd_kv_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                  const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
+                  AttnParams p) {
+  constexpr int TILE = 32 * D;
+  constexpr int NT = D / 8;
+  constexpr int HALVES = D / 64;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* sm = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  __shared__ __align__(8) uint64_t bars_all[kKVWarps][1 + kRing];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int bh = blockIdx.y;
+  const int n1 = p.N >> 4;
+  const int c = blockIdx.x * kKVWarps + warp;  // key block
+  const bool active = c < n1;
+  const int K = p.K;
+
+  const uint32_t w0 = smem_u32(sm + (size_t)warp * TILE * (2 + 2 * kRing));
+  const uint32_t kt = w0, vt = w0 + TILE;
+  auto ring_q = [&](int st) { return w0 + (uint32_t)(2 + 2 * st) * TILE; };
+  auto ring_do = [&](int st) { return w0 + (uint32_t)(3 + 2 * st) * TILE; };
+  const uint32_t bar0 = smem_u32(&bars_all[warp][0]);
+  auto bar_of = [&](int st) { return bar0 + 8u * (1 + st); };
+  if (lane == 0) {
+    for (int i = 0; i <= kRing; ++i) mbar_init(bar0 + 8u * i, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  if (!active) return;
+
+  const size_t rowbase = (size_t)bh * p.N;
+  const int32_t* rp = p.row_ptr[1] + (size_t)bh * (n1 + 1);
+  const int32_t* col = p.col[1] + (size_t)bh * n1 * K;
+  const int beg = rp[c];
+  const int nq = rp[c + 1] - beg;
+  auto issue = [&](int r) {
+    if (lane == 0) {
+      const int qb = col[beg + r];
+      const int st = r % kRing;
+      mbar_arrive_expect_tx(bar_of(st), 2u * TILE);
+      const int y = (int)(rowbase + (size_t)qb * 16);
+#pragma unroll
+      for (int h = 0; h < HALVES; ++h) {
+        tma_load_2d(ring_q(st) + h * 2048, &tq, 64 * h, y, bar_of(st));
+        tma_load_2d(ring_do(st) + h * 2048, &tdo, 64 * h, y, bar_of(st));
+      }
+    }
+  };
+  if (lane == 0) {
+    mbar_arrive_expect_tx(bar0, 2u * TILE);
+    const int y = (int)(rowbase + (size_t)c * 16);
+#pragma unroll
+    for (int h = 0; h < HALVES; ++h) {
+      tma_load_2d(kt + h * 2048, &tk, 64 * h, y, bar0);
+      tma_load_2d(vt + h * 2048, &tv, 64 * h, y, bar0);
+    }
+  }
+  for (int r = 0; r < nq && r < kRing; ++r) issue(r);
+
+  bool ok = mbar_wait_bounded(bar0, 0);
+  uint32_t ka[D / 16][4], va[D / 16][4];
+  load_a_frags<D>(kt, lane, ka);
+  load_a_frags<D>(vt, lane, va);
+  float dk[NT][4], dv[NT][4];
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    dk[nt][0] = dk[nt][1] = dk[nt][2] = dk[nt][3] = 0.f;
+    dv[nt][0] = dv[nt][1] = dv[nt][2] = dv[nt][3] = 0.f;
+  }
+  const float sc2 = p.scale * kLog2e;
+  int r = 0;
+  for (; r < nq && ok; ++r) {
+    const int st = r % kRing;
+    const int qb = col[beg + r];
+    // LSE and Delta of the queries in this thread's columns: 2t, 2t+1, 8+2t, 9+2t
+    const size_t q0 = rowbase + (size_t)qb * 16;
+    float lse[2][2], dl[2][2];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        lse[nt][e] = p.lse_in[q0 + 8 * nt + 2 * t + e] * kLog2e;
+        dl[nt][e] = p.delta[q0 + 8 * nt + 2 * t + e];
+      }
+    ok = mbar_wait_bounded(bar_of(st), (uint32_t)((r / kRing) & 1));
+    if (!ok) break;
+    float s[2][4], dpv[2][4], P[2][4], dS[2][4];
+    qk_tile<D>(ka, ring_q(st), lane, s);    // S^T: rows keys, columns queries
+    qk_tile<D>(va, ring_do(st), lane, dpv); // dP^T
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float l2 = lse[nt][e & 1];
+        P[nt][e] = (l2 == -INFINITY) ? 0.f : exp2f(fmaf(s[nt][e], sc2, -l2));
+        dS[nt][e] = P[nt][e] * (dpv[nt][e] - dl[nt][e & 1]);
+      }
+    uint32_t ph[4], pl[4], dsh[4], dsl[4];
+    split_frag(P, ph, pl);
+    split_frag(dS, dsh, dsl);
+    pv_tile2<D>(ph, pl, ring_do(st), lane, dv);
+    pv_tile2<D>(dsh, dsl, ring_q(st), lane, dk);
+    __syncwarp();
+    fence_proxy_async_smem();
+    if (r + kRing < nq) issue(r + kRing);
+  }
+  if (!ok) {
+    for (int q = r; q < nq && q < r + kRing; ++q)
+      mbar_wait_bounded(bar_of(q % kRing), (uint32_t)((q / kRing) & 1));
+    if (lane == 0) report_status(p.status, LLSA_DEV_TIMEOUT);
+    return;
+  }
+  // epilogue: dK = scale * acc + sum_l coarse dK(l)[t >> 4l] / 16^l (likewise dV)
+  bf16* dK = static_cast<bf16*>(p.dk);
+  bf16* dV = static_cast<bf16*>(p.dv);
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const size_t tok = (size_t)c * 16 + g + 8 * half;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int d = 8 * nt + 2 * t;
+      float k0 = dk[nt][2 * half] * p.scale, k1 = dk[nt][2 * half + 1] * p.scale;
+      float v0 = dv[nt][2 * half], v1 = dv[nt][2 * half + 1];
+      for (int l = 2; l <= p.L; ++l) {
+        const float inv = 1.0f / (float)(1u << (4 * l));
+        const float* cg = p.coarse[l] + ((size_t)bh * (p.N >> (4 * l)) + (tok >> (4 * l))) * 2 * D;
+        const float2 gk = *reinterpret_cast<const float2*>(cg + d);
+        const float2 gv = *reinterpret_cast<const float2*>(cg + D + d);
+        k0 += gk.x * inv;
+        k1 += gk.y * inv;
+        v0 += gv.x * inv;
+        v1 += gv.y * inv;
+      }
+      *reinterpret_cast<uint32_t*>(dK + (rowbase + tok) * D + d) = pack_bf16(k0, k1);
+      *reinterpret_cast<uint32_t*>(dV + (rowbase + tok) * D + d) = pack_bf16(v0, v1);
+    }
+  }
+}
+
+template <int D>
+cudaError_t launch_typed(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s) {
+  constexpr int TILE = 32 * D;
+  const int BH = p.B * p.H;
+  const int n1 = p.N / kBlock;
+  const int nct = ((p.L - 1) * p.K + 15) / 16;
+  // pass 1
+  const size_t smem1 = 1024 + (size_t)kQWarps * TILE * 2 * kRing + 2 * (size_t)nct * TILE +
+                       nct * 16 * sizeof(float) + kQWarps * (1 + kRing) * 8 + 2 * nct * 16 * sizeof(int);
+  cudaError_t e = cudaFuncSetAttribute(bwd_q_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
+  if (e != cudaSuccess) return e;
+  bwd_q_mma_kernel<D><<<dim3((n1 + kQWarps - 1) / kQWarps, BH), kQWarps * 32, smem1, s>>>(
+      maps[0], maps[1], maps[2], maps[3], p, nct);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // pass 2
+  e = launch_coarse_reduce(p, s);
+  if (e != cudaSuccess) return e;
+  // pass 3
+  const size_t smem3 = 1024 + (size_t)kKVWarps * TILE * (2 + 2 * kRing);
+  e = cudaFuncSetAttribute(bwd_kv_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3);
+  if (e != cudaSuccess) return e;
+  bwd_kv_mma_kernel<D><<<dim3((n1 + kKVWarps - 1) / kKVWarps, BH), kKVWarps * 32, smem3, s>>>(
+      maps[0], maps[1], maps[2], maps[3], p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+// maps: Q, K, V, dO as 2D [B*H*N rows, D cols] bf16 tile maps (16 x 64, 128B swizzle).
+cudaError_t launch_attn_bwd_mma(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s) {
+  return (p.D == 64) ? launch_typed<64>(p, maps, s) : launch_typed<128>(p, maps, s);
+}
+
+}  // namespace llsa

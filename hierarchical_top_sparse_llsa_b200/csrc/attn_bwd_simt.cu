@@ -4,8 +4,8 @@
 // Transformers"; Building Blocks: Sparse Index Transpose).
 //
 // Three launches, no global atomics, every sum in a fixed order:
-//   1. query-major: one CTA per level-2 token (16 query blocks that share
-//      every coarse key set; one CTA per block when L = 1).  It forms
+//   1. query-major: one CTA per 8 consecutive query blocks (they share every
+//      coarse key set; one CTA per block when L = 1).  It forms
 //      Delta_i = sum_j P_ij dP_ij (equal to dO_i . O_i, but taken from the
 //      unrounded terms: O itself is stored rounded to its dtype), dQ, and the
 //      coarse-key partials
@@ -47,7 +47,7 @@ bwd_query_simt_kernel(AttnParams p, int G) {
   const int tid = threadIdx.x;
   const int i = tid >> 4, sub = tid & 15;
   const int K = p.K;
-  const int N2 = p.N >> 8;
+  const int NG = p.N >> 7;  // partial groups of 8 query blocks per (b, h)
   const T* Q = static_cast<const T*>(p.q);
   const T* Kf = static_cast<const T*>(p.k);
   const T* Vf = static_cast<const T*>(p.v);
@@ -76,7 +76,7 @@ bwd_query_simt_kernel(AttnParams p, int G) {
 
   // zero this CTA's partial slots (levels 2..L)
   for (int l = 2; l <= p.L; ++l) {
-    float* part = p.part[l] + ((size_t)bh * N2 + g) * K * 2 * D;
+    float* part = p.part[l] + ((size_t)bh * NG + g) * K * 2 * D;
     for (int e = tid; e < K * 2 * D; e += 256) part[e] = 0.f;
   }
   int flags = 0;
@@ -178,7 +178,7 @@ bwd_query_simt_kernel(AttnParams p, int G) {
           gk = fmaf(dss[r][j], qs[r][d], gk);
           gv = fmaf(ps[r][j], dos[r][d], gv);
         }
-        float* part = p.part[lv] + (((size_t)bh * N2 + g) * K + kl.slot[t0 + j]) * 2 * D;
+        float* part = p.part[lv] + (((size_t)bh * NG + g) * K + kl.slot[t0 + j]) * 2 * D;
         part[d] += gk * p.scale;
         part[D + d] += gv;
       }
@@ -196,8 +196,8 @@ __global__ void bwd_coarse_reduce_kernel(AttnParams p, int l) {
   const int bh = blockIdx.y;
   const int D = p.D, K = p.K;
   const int nl = p.N >> (4 * l);
-  const int N2 = p.N >> 8;
-  const int span2 = 1 << (4 * (l - 2));  // level-2 descendants of a level-l token
+  const int NG = p.N >> 7;
+  const int span = 2 << (4 * (l - 2));   // groups of 8 query blocks under a level-l token
   const int t = threadIdx.x;             // kv * D + d
   const int32_t* rp = p.row_ptr[l] + (size_t)bh * (nl + 1);
   const int32_t* col = p.col[l] + (size_t)bh * nl * K;
@@ -210,9 +210,9 @@ __global__ void bwd_coarse_reduce_kernel(AttnParams p, int l) {
     for (int s = 0; s < K; ++s)
       if (rr.use(row[s], nl) && row[s] == c) slot = s;
     if (slot < 0) continue;
-    for (int a = 0; a < span2; ++a) {
-      const size_t a2 = (size_t)ql * span2 + a;
-      acc += p.part[l][(((size_t)bh * N2 + a2) * K + slot) * 2 * D + t];
+    for (int a = 0; a < span; ++a) {
+      const size_t grp = (size_t)ql * span + a;
+      acc += p.part[l][(((size_t)bh * NG + grp) * K + slot) * 2 * D + t];
     }
   }
   p.coarse[l][((size_t)bh * nl + c) * 2 * D + t] = acc;
@@ -317,20 +317,26 @@ template <typename T, int D>
 cudaError_t launch_typed(const AttnParams& p, cudaStream_t s) {
   const int BH = p.B * p.H;
   const int n1 = p.N / kBlock;
-  const int G = (p.L >= 2) ? 16 : 1;
+  const int G = (p.L >= 2) ? 8 : 1;
   bwd_query_simt_kernel<T, D><<<dim3(n1 / G, BH), 256, 0, s>>>(p, G);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  for (int l = 2; l <= p.L; ++l) {
-    bwd_coarse_reduce_kernel<<<dim3(p.N >> (4 * l), BH), 2 * D, 0, s>>>(p, l);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-  }
+  e = launch_coarse_reduce(p, s);
+  if (e != cudaSuccess) return e;
   bwd_kv_simt_kernel<T, D><<<dim3(n1, BH), 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 
 }  // namespace
+
+cudaError_t launch_coarse_reduce(const AttnParams& p, cudaStream_t s) {
+  for (int l = 2; l <= p.L; ++l) {
+    bwd_coarse_reduce_kernel<<<dim3(p.N >> (4 * l), p.B * p.H), 2 * p.D, 0, s>>>(p, l);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
 
 cudaError_t launch_attn_bwd_simt(const AttnParams& p, int dtype, cudaStream_t s) {
   if (dtype == LLSA_BF16)

@@ -17,7 +17,7 @@
 #include <math.h>
 
 #include "keyset.cuh"
-#include "sm100_ptx.cuh"
+#include "mma_tiles.cuh"
 
 namespace llsa {
 
@@ -83,43 +83,6 @@ __device__ __forceinline__ void softmax_tile(float (&s)[2][4], const float (&lw)
   pa[1] = pack_bf16(p[0][2], p[0][3]);
   pa[2] = pack_bf16(p[1][0], p[1][1]);
   pa[3] = pack_bf16(p[1][2], p[1][3]);
-}
-
-// S (16 x 16) = Q (16 x D, A fragments) . K_tile^T; the K tile is a swizzled
-// 16-row tile at `kt` (shared address).
-template <int D>
-__device__ __forceinline__ void qk_tile(const uint32_t (&qa)[D / 16][4], uint32_t kt, int lane,
-                                        float (&s)[2][4]) {
-  const int mi = lane >> 3;
-  const int krow = (mi >> 1) * 8 + (lane & 7);
-  const int kc = mi & 1;
-#pragma unroll
-  for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
-#pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    uint32_t b0, b1, b2, b3;
-    ldsm_x4(kt + swz(krow, 2 * kk + kc), b0, b1, b2, b3);
-    mma_bf16(s[0], qa[kk], b0, b1);
-    mma_bf16(s[1], qa[kk], b2, b3);
-  }
-}
-
-// O (16 x D) += P (16 x 16, A fragment) . V_tile (16 x D, swizzled at vt).
-template <int D>
-__device__ __forceinline__ void pv_tile(const uint32_t (&pa)[4], uint32_t vt, int lane,
-                                        float (&o)[D / 8][4]) {
-  const int mi = lane >> 3;
-  const int vrow = (mi & 1) * 8 + (lane & 7);
-  const int vc = mi >> 1;
-#pragma unroll
-  for (int nn = 0; nn < D / 16; ++nn) {
-    uint32_t b0, b1, b2, b3;
-    ldsm_x4_t(vt + swz(vrow, 2 * nn + vc), b0, b1, b2, b3);
-    mma_bf16(o[2 * nn], pa, b0, b1);
-    mma_bf16(o[2 * nn + 1], pa, b2, b3);
-  }
 }
 
 template <int D>

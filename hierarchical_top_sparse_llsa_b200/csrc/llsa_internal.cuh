@@ -141,7 +141,7 @@ struct AttnParams {
   void* dk;
   void* dv;
   float* delta;                 // [BH, N]
-  float* part[kMaxL + 1];       // [BH, N_2, K, 2, D] per coarse level
+  float* part[kMaxL + 1];       // [BH, N/128, K, 2, D] per coarse level (groups of 8 query blocks)
   float* coarse[kMaxL + 1];     // [BH, N_l, 2, D] per coarse level
   int32_t* status;
   int B, H, N, D, L, K;
@@ -153,6 +153,6 @@ struct AttnParams {
 cudaError_t launch_pool(const PoolParams& p, int dtype, cudaStream_t s);
 cudaError_t launch_select_level(const SelectParams& p, int BH, int D, cudaStream_t s);
 cudaError_t launch_transpose(const TransposeParams& p, cudaStream_t s);
-cudaError_t launch_attn_bwd(const AttnParams& p, int dtype, cudaStream_t s);
+cudaError_t launch_coarse_reduce(const AttnParams& p, cudaStream_t s);
 
 }  // namespace llsa

@@ -179,7 +179,9 @@ LLSA_API size_t llsa_bwd_workspace_bytes(const llsa_desc* desc);
  *   is spread to each of its 16^l fine tokens divided by 16^l (the mean's
  *   derivative).  Selection passes no gradient.  Sums run in a fixed order
  *   without global atomics, so results are identical from run to run.
- *   o, lse: the outputs of llsa_attn_fwd.  dout: dO.  csr: llsa_index_transpose
+ *   o, lse: the outputs of llsa_attn_fwd (o must be valid but is not read:
+ *   Delta_i = sum_j P_ij (dO_i . v_j) is recomputed from unrounded terms, as O
+ *   itself is stored rounded to dtype).  dout: dO.  csr: llsa_index_transpose
  *   of the same idx.  dq, dk, dv: [B, H, N, D] dtype, written.
  *   ws: device scratch of at least llsa_bwd_workspace_bytes(desc) bytes,
  *   256-byte aligned.  dev_status: may be NULL.

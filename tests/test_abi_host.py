@@ -85,7 +85,7 @@ def test_workspace_size_and_checks(lib):
     B, H, N, D, L, K = 1, 2, 4096, 64, 3, 8
     r256 = lambda x: (x + 255) // 256 * 256
     want = r256(B * H * N * 4)
-    want += sum(r256(B * H * (N // 256) * K * 2 * D * 4) for _ in range(2, L + 1))
+    want += sum(r256(B * H * (N // 128) * K * 2 * D * 4) for _ in range(2, L + 1))
     want += sum(r256(B * H * (N // 16**l) * 2 * D * 4) for l in range(2, L + 1))
     assert llsa.llsa_bwd_workspace_bytes(d) == want
     # fill every pointer with a fake non-null value: the size check fails first
