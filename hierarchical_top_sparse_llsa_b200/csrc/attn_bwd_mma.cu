@@ -10,10 +10,11 @@
 //   sweep 1: S = Q K^T, dP = dO V^T, P = w e^{S - LSE}, Delta_i = sum_j P dP
 //            (from unrounded terms: O is stored rounded);
 //   sweep 2: dS = P (dP - Delta), dQ += dS K.
-// P and dS enter their MMAs as a bf16 hi + lo pair (about 16 mantissa bits):
-// the sums over queries in dK and dV cancel strongly on image-like inputs,
-// and single bf16 rounding of dS left some small dK entries 3x outside a
-// 2e-2 relative band.
+// In the sums over queries (dK, dV and the coarse partials) P and dS enter
+// their MMAs as a bf16 hi + lo pair (about 16 mantissa bits): those sums
+// cancel strongly on image-like inputs, and single bf16 rounding left some
+// small dK entries 3x (dV 1.5x) outside a 2e-2 relative band.  dQ, a sum
+// over keys, keeps a single bf16 dS (worst case 0.45 of that band).
 // Coarse keys then give dQ their share and, per CTA, the partials
 // sum_i dS_ij q_i and sum_i P_ij dO_i: each warp forms its block's part with
 // MMAs on register transposes (movmatrix), and the CTA adds the 8 parts in a
@@ -127,13 +128,9 @@ bwd_q_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
   auto bar_of = [&](int st) { return bar0 + 8u * (1 + st); };
 
   int flags = 0;
-  int my_blk = -1;
-  bool used = false;
-  if (active && lane < K) {
-    const int32_t* row = p.idx[1] + ((size_t)bh * n1 + b) * K;
-    used = row_entry_used(row, lane, n1, flags);
-    my_blk = row[lane];
-  }
+  const bool on_row = active && lane < K;
+  const int my_blk = on_row ? p.idx[1][((size_t)bh * n1 + b) * K + lane] : -1;
+  const bool used = warp_row_used(my_blk, lane, n1, on_row, flags);
   const unsigned fmask = __ballot_sync(0xffffffffu, used);
   const int nf = __popc(fmask);
   if (used) flist[__popc(fmask & ((1u << lane) - 1u))] = my_blk;
@@ -145,13 +142,8 @@ bwd_q_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
     for (int l = 2; l <= p.L; ++l) {
       const int nl = p.N >> (4 * l);
       const int a = b0 >> (4 * (l - 1));
-      bool u = false;
-      int c = -1;
-      if (lane < K) {
-        const int32_t* row = p.idx[l] + ((size_t)bh * nl + a) * K;
-        u = row_entry_used(row, lane, nl, flags);
-        c = row[lane];
-      }
+      const int c = (lane < K) ? p.idx[l][((size_t)bh * nl + a) * K + lane] : -1;
+      const bool u = warp_row_used(c, lane, nl, lane < K, flags);
       const unsigned m = __ballot_sync(0xffffffffu, u);
       if (u) {
         const int pos = n + __popc(m & ((1u << lane) - 1u));
@@ -293,9 +285,9 @@ bwd_q_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) P[nt][e] *= dpv[nt][e] - ((e < 2) ? delta_g : delta_g8);
-      uint32_t dsh[4], dsl[4];
-      split_frag(P, dsh, dsl);
-      pv_tile2<D>(dsh, dsl, ring_k(st), lane, dq);
+      uint32_t dsa[4];
+      pack_frag(P, dsa);
+      pv_tile<D>(dsa, ring_k(st), lane, dq);
       __syncwarp();
       fence_proxy_async_smem();
       if (r + kRing < ntiles) issue(r + kRing);

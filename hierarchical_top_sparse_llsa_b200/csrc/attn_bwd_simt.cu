@@ -190,29 +190,53 @@ bwd_query_simt_kernel(AttnParams p, int G) {
   }
 }
 
-// Coarse gradient of token c at level l: thread per (kv, d).
+// Coarse gradient of token c at level l: thread per (kv, d).  The (query
+// token, slot) pairs of row c of the level-l key-major lists are found first,
+// in parallel, then every thread sums its column over them in order.
+constexpr int kReduceChunk = 128;
 __global__ void bwd_coarse_reduce_kernel(AttnParams p, int l) {
+  __shared__ int s_q[kReduceChunk], s_slot[kReduceChunk];
   const int c = blockIdx.x;
   const int bh = blockIdx.y;
   const int D = p.D, K = p.K;
   const int nl = p.N >> (4 * l);
   const int NG = p.N >> 7;
-  const int span = 2 << (4 * (l - 2));   // groups of 8 query blocks under a level-l token
-  const int t = threadIdx.x;             // kv * D + d
+  const int span = 2 << (4 * (l - 2));  // groups of 8 query blocks under a level-l token
+  const int t = threadIdx.x;            // kv * D + d
   const int32_t* rp = p.row_ptr[l] + (size_t)bh * (nl + 1);
   const int32_t* col = p.col[l] + (size_t)bh * nl * K;
+  const float* part = p.part[l] + (size_t)bh * NG * K * 2 * D + t;
+  const int beg = rp[c], end = rp[c + 1];
   float acc = 0.f;
-  for (int e = rp[c]; e < rp[c + 1]; ++e) {
-    const int ql = col[e];
-    const int32_t* row = p.idx[l] + ((size_t)bh * nl + ql) * K;
-    RowRule rr;
-    int slot = -1;
-    for (int s = 0; s < K; ++s)
-      if (rr.use(row[s], nl) && row[s] == c) slot = s;
-    if (slot < 0) continue;
-    for (int a = 0; a < span; ++a) {
-      const size_t grp = (size_t)ql * span + a;
-      acc += p.part[l][(((size_t)bh * NG + grp) * K + slot) * 2 * D + t];
+  for (int e0 = beg; e0 < end; e0 += kReduceChunk) {
+    const int cnt = min(kReduceChunk, end - e0);
+    __syncthreads();
+    for (int e = t; e < cnt; e += blockDim.x) {
+      const int ql = col[e0 + e];
+      const int32_t* row = p.idx[l] + ((size_t)bh * nl + ql) * K;
+      RowRule rr;
+      int slot = -1;
+      for (int s = 0; s < K; ++s)
+        if (rr.use(row[s], nl) && row[s] == c) slot = s;
+      s_q[e] = ql;
+      s_slot[e] = slot;
+    }
+    __syncthreads();
+    for (int e = 0; e < cnt; ++e) {
+      const int slot = s_slot[e];
+      if (slot < 0) continue;
+      const float* src = part + ((size_t)s_q[e] * span * K + slot) * 2 * D;
+      const size_t stride = (size_t)K * 2 * D;  // next group, same slot
+      int a = 0;
+      for (; a + 4 <= span; a += 4) {
+        const float x0 = src[(a + 0) * stride], x1 = src[(a + 1) * stride];
+        const float x2 = src[(a + 2) * stride], x3 = src[(a + 3) * stride];
+        acc += x0;
+        acc += x1;
+        acc += x2;
+        acc += x3;
+      }
+      for (; a < span; ++a) acc += src[a * stride];
     }
   }
   p.coarse[l][((size_t)bh * nl + c) * 2 * D + t] = acc;

@@ -6,8 +6,10 @@
 // One warp owns one 16-token query block (the block is exactly the M = 16 of
 // the warp MMA).  Its selected 16-token key blocks are contiguous 16-row
 // tiles of K and V, gathered by 2D TMA loads (128-byte swizzle, no
-// multicast) into a 3-stage ring with one mbarrier per stage, so the next
-// tiles are in flight while the current one is multiplied.  A CTA holds 4
+// multicast) into a 2-stage ring with one mbarrier per stage (the Q tile
+// passes through stage 0 first); S of the next tile is issued before the
+// softmax and PV of the current one, so the MMA pipe has work while the
+// exponentials run.  A CTA holds 4
 // sibling query blocks (same level-2 ancestor), which share every coarse
 // key; the coarse K/V rows (fp32 pyramid) are converted once per CTA to bf16
 // tiles in shared memory, with ln(w_l) per key folded into the scores.
@@ -24,7 +26,7 @@ namespace llsa {
 namespace {
 
 constexpr int kFwdWarps = 4;
-constexpr int kStages = 3;
+constexpr int kStages = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -103,8 +105,8 @@ attn_fwd_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
   const bool active = b < n1;
   const int K = p.K;
 
-  unsigned char* wbase = sm + (size_t)warp * TILE * (1 + 2 * kStages);
-  unsigned char* ck = sm + (size_t)kFwdWarps * TILE * (1 + 2 * kStages);
+  unsigned char* wbase = sm + (size_t)warp * TILE * 2 * kStages;
+  unsigned char* ck = sm + (size_t)kFwdWarps * TILE * 2 * kStages;
   unsigned char* cv = ck + (size_t)nct * TILE;
   float* clw = reinterpret_cast<float*>(cv + (size_t)nct * TILE);
   uint64_t* bars = reinterpret_cast<uint64_t*>(clw + nct * 16);
@@ -113,21 +115,17 @@ attn_fwd_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
   __shared__ int flist_all[kFwdWarps][32];  // each warp's used fine blocks, ascending
   int* flist = flist_all[warp];
 
-  const uint32_t qt = smem_u32(wbase);
+  const uint32_t w0 = smem_u32(wbase);
   const uint32_t bar0 = smem_u32(bars + warp * (kStages + 1));  // [0] = Q, [1..] = stages
-  auto stage_k = [&](int st) { return qt + (uint32_t)(1 + 2 * st) * TILE; };
-  auto stage_v = [&](int st) { return qt + (uint32_t)(2 + 2 * st) * TILE; };
+  auto stage_k = [&](int st) { return w0 + (uint32_t)(2 * st) * TILE; };
+  auto stage_v = [&](int st) { return w0 + (uint32_t)(2 * st + 1) * TILE; };
   auto bar_of = [&](int st) { return bar0 + 8u * (1 + st); };
 
   int flags = 0;
   // ---- this warp's fine blocks (lane s holds slot s of its row of I(1))
-  int my_blk = -1;
-  bool used = false;
-  if (active && lane < K) {
-    const int32_t* row = p.idx[1] + ((size_t)bh * n1 + b) * K;
-    used = row_entry_used(row, lane, n1, flags);
-    my_blk = row[lane];
-  }
+  const bool on_row = active && lane < K;
+  const int my_blk = on_row ? p.idx[1][((size_t)bh * n1 + b) * K + lane] : -1;
+  const bool used = warp_row_used(my_blk, lane, n1, on_row, flags);
   const unsigned fmask = __ballot_sync(0xffffffffu, used);
   const int nf = __popc(fmask);
   if (used) flist[__popc(fmask & ((1u << lane) - 1u))] = my_blk;
@@ -140,13 +138,8 @@ attn_fwd_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
     for (int l = 2; l <= p.L; ++l) {
       const int nl = p.N >> (4 * l);
       const int a = b0 >> (4 * (l - 1));
-      bool u = false;
-      int c = -1;
-      if (lane < K) {
-        const int32_t* row = p.idx[l] + ((size_t)bh * nl + a) * K;
-        u = row_entry_used(row, lane, nl, flags);
-        c = row[lane];
-      }
+      const int c = (lane < K) ? p.idx[l][((size_t)bh * nl + a) * K + lane] : -1;
+      const bool u = warp_row_used(c, lane, nl, lane < K, flags);
       const unsigned m = __ballot_sync(0xffffffffu, u);
       if (u) clist[n + __popc(m & ((1u << lane) - 1u))] = (l << 24) | c;
       n += __popc(m);
@@ -181,7 +174,7 @@ attn_fwd_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
   for (int e = threadIdx.x; e < ncpad * 16; e += blockDim.x)
     clw[e] = (e < nc) ? p.logw[clist[e] >> 24] * kLog2e : -INFINITY;
 
-  // ---- issue Q and the first fine tiles
+  // ---- Q lands in stage 0 first; the fine tiles follow once its fragments are read
   const size_t rowbase = (size_t)bh * p.N;
   auto issue_block = [&](int r) {
     if (lane == 0) {
@@ -200,22 +193,21 @@ attn_fwd_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
     if (lane == 0) {
       mbar_arrive_expect_tx(bar0, TILE);
 #pragma unroll
-      for (int h = 0; h < HALVES; ++h) tma_load_2d(qt + h * 2048, &tq, 64 * h, (int)(rowbase + (size_t)b * 16), bar0);
+      for (int h = 0; h < HALVES; ++h)
+        tma_load_2d(stage_k(0) + h * 2048, &tq, 64 * h, (int)(rowbase + (size_t)b * 16), bar0);
     }
-    for (int r = 0; r < nf && r < kStages; ++r) issue_block(r);
+    if (nf > 1) issue_block(1);  // stage 1 is free; stage 0 holds Q for now
   }
   __syncthreads();  // coarse tiles written
   if (!active) return;
 
   bool ok = mbar_wait_bounded(bar0, 0);
   uint32_t qa[D / 16][4];
-  {
-    const int mi = lane >> 3;
-    const int row = (mi & 1) * 8 + (lane & 7);
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk)
-      ldsm_x4(qt + swz(row, 2 * kk + (mi >> 1)), qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
-  }
+  load_a_frags<D>(stage_k(0), lane, qa);
+  __syncwarp();
+  fence_proxy_async_smem();
+  if (nf > 0) issue_block(0);
+
   float o[NT][4];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
@@ -225,19 +217,34 @@ attn_fwd_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
   const float sc2 = p.scale * kLog2e;
   const float zero_lw[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 
+  // software pipeline: S of tile r+1 is issued before the softmax and PV of tile r
+  float s_cur[2][4];
   int r = 0;
+  if (nf > 0 && ok) {
+    ok = mbar_wait_bounded(bar_of(0), 0);
+    if (ok) qk_tile<D>(qa, stage_k(0), lane, s_cur);
+  }
   for (; r < nf && ok; ++r) {
     const int sidx = r % kStages;
-    ok = mbar_wait_bounded(bar_of(sidx), (uint32_t)((r / kStages) & 1));
-    if (!ok) break;
-    float s[2][4];
+    float s_next[2][4];
+    if (r + 1 < nf) {
+      const int nidx = (r + 1) % kStages;
+      ok = mbar_wait_bounded(bar_of(nidx), (uint32_t)(((r + 1) / kStages) & 1));
+      if (!ok) break;
+      qk_tile<D>(qa, stage_k(nidx), lane, s_next);
+    }
     uint32_t pa[4];
-    qk_tile<D>(qa, stage_k(sidx), lane, s);
-    softmax_tile<NT>(s, zero_lw, sc2, st, o, pa);
+    softmax_tile<NT>(s_cur, zero_lw, sc2, st, o, pa);
     pv_tile<D>(pa, stage_v(sidx), lane, o);
     __syncwarp();
     fence_proxy_async_smem();
     if (r + kStages < nf) issue_block(r + kStages);
+    if (r + 1 < nf) {
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s_cur[a][e] = s_next[a][e];
+    }
   }
   if (!ok) {
     // give the copies already in flight a bounded chance to land, then stop
@@ -287,7 +294,7 @@ template <int D>
 cudaError_t launch_typed(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s) {
   constexpr int TILE = 32 * D;
   const int nct = ((p.L - 1) * p.K + 15) / 16;
-  const size_t smem = 1024 + (size_t)kFwdWarps * TILE * (1 + 2 * kStages) + 2 * (size_t)nct * TILE +
+  const size_t smem = 1024 + (size_t)kFwdWarps * TILE * 2 * kStages + 2 * (size_t)nct * TILE +
                       nct * 16 * sizeof(float) + kFwdWarps * (kStages + 1) * 8 + nct * 16 * sizeof(int);
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_mma_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

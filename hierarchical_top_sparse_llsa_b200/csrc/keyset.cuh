@@ -28,13 +28,8 @@ __device__ __forceinline__ int build_key_list(KeyList& kl, const AttnParams& p, 
   int n = 0;
   {
     const int n1 = p.N / kBlock;
-    const int32_t* row = p.idx[1] + ((size_t)bh * n1 + b) * K;
-    bool u = false;
-    int c = -1;
-    if (lane < K) {
-      u = row_entry_used(row, lane, n1, flags);
-      c = row[lane];
-    }
+    const int c = (lane < K) ? p.idx[1][((size_t)bh * n1 + b) * K + lane] : -1;
+    const bool u = warp_row_used(c, lane, n1, lane < K, flags);
     const unsigned m = __ballot_sync(0xffffffffu, u);
     if (u) {
       const int pos = __popc(m & ((1u << lane) - 1u)) * kBlock;
@@ -50,13 +45,8 @@ __device__ __forceinline__ int build_key_list(KeyList& kl, const AttnParams& p, 
   for (int l = 2; l <= p.L; ++l) {
     const int nl = p.N >> (4 * l);
     const int a = b >> (4 * (l - 1));
-    const int32_t* row = p.idx[l] + ((size_t)bh * nl + a) * K;
-    bool u = false;
-    int c = -1;
-    if (lane < K) {
-      u = row_entry_used(row, lane, nl, flags);
-      c = row[lane];
-    }
+    const int c = (lane < K) ? p.idx[l][((size_t)bh * nl + a) * K + lane] : -1;
+    const bool u = warp_row_used(c, lane, nl, lane < K, flags);
     const unsigned m = __ballot_sync(0xffffffffu, u);
     if (u) {
       const int pos = n + __popc(m & ((1u << lane) - 1u));

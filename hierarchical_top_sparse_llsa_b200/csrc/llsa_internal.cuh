@@ -74,16 +74,38 @@ struct RowRule {
   }
 };
 
-// Used flag of entry `s` of a row (the row rule applied to the row's prefix).
-__device__ __forceinline__ bool row_entry_used(const int32_t* row, int s, int n, int& flags) {
-  RowRule rr;
-  bool u = false;
-  for (int t = 0; t <= s; ++t) {
-    const int f0 = rr.flags;
-    u = rr.use(row[t], n);
-    if (t == s) flags |= rr.flags & ~f0;
+// The same rule for rows laid side by side across a warp: this lane holds
+// entry `slot` of a row whose entry 0 sits `slot` lanes lower; `on` is false
+// for lanes outside every row (their results are ignored and they are never
+// read by lanes inside a row).  Segmented shuffle scans give, for each entry,
+// the largest in-range entry before it and whether a pad came before it.
+// Must be called by all 32 lanes.
+__device__ __forceinline__ bool warp_row_used(int v, int slot, int n, bool on, int& flags) {
+  const bool inr = on && v >= 0 && v < n;
+  int mx = inr ? v : -1;
+  int pad = (on && v == -1) ? 1 : 0;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, mx, o);
+    const int z = __shfl_up_sync(0xffffffffu, pad, o);
+    if (slot >= o) {
+      mx = max(mx, y);
+      pad |= z;
+    }
   }
-  return u;
+  int mx_before = __shfl_up_sync(0xffffffffu, mx, 1);
+  int pad_before = __shfl_up_sync(0xffffffffu, pad, 1);
+  if (slot < 1) {
+    mx_before = -1;
+    pad_before = 0;
+  }
+  const bool used = inr && v > mx_before;
+  if (on) {
+    if (v < -1 || v >= n) flags |= LLSA_DEV_BAD_INDEX;
+    else if (inr && !used) flags |= LLSA_DEV_NONCANONICAL;
+    else if (used && pad_before) flags |= LLSA_DEV_NONCANONICAL;
+  }
+  return used;
 }
 
 __device__ __forceinline__ void report_status(int32_t* st, int flags) {

@@ -53,8 +53,9 @@ transpose_kernel(TransposeParams p) {
   __syncthreads();
 
   const int rows_per_step = 32 / K;  // K <= 32
-  const int sub = lane / K, slot = lane % K;
+  const int sub = lane / K;
   const bool lane_on = sub < rows_per_step;
+  const int slot = lane_on ? lane % K : lane;  // lanes past the last row never feed a row
   const int rpw = (n + kTrWarps - 1) / kTrWarps;  // rows per warp
   const int r_begin = min(n, warp * rpw), r_end = min(n, r_begin + rpw);
 
@@ -62,13 +63,11 @@ transpose_kernel(TransposeParams p) {
   int flags = 0, my_below = 0;
   for (int r0 = r_begin; r0 < r_end; r0 += rows_per_step) {
     const int q = r0 + sub;
-    if (lane_on && q < r_end) {
-      const int32_t* row = I + (size_t)q * K;
-      const bool u = row_entry_used(row, slot, n, flags);
-      const int c = row[slot];
-      if (u && c >= c0 && c < c1) atomicAdd(&hist[warp][c - c0], 1);
-      if (u && c < c0) ++my_below;
-    }
+    const bool on = lane_on && q < r_end;
+    const int c = on ? I[(size_t)q * K + slot] : -1;
+    const bool u = warp_row_used(c, slot, n, on, flags);
+    if (u && c >= c0 && c < c1) atomicAdd(&hist[warp][c - c0], 1);
+    if (u && c < c0) ++my_below;
   }
   my_below = __reduce_add_sync(0xffffffffu, my_below);
   if (lane == 0) below[warp] = my_below;
@@ -120,13 +119,10 @@ transpose_kernel(TransposeParams p) {
   int dummy = 0;
   for (int r0 = r_begin; r0 < r_end; r0 += rows_per_step) {
     const int q = r0 + sub;
-    int key = -2 - lane;  // unique per lane: matches nobody
-    if (lane_on && q < r_end) {
-      const int32_t* row = I + (size_t)q * K;
-      const bool u = row_entry_used(row, slot, n, dummy);
-      const int c = row[slot];
-      if (u && c >= c0 && c < c1) key = c;
-    }
+    const bool on = lane_on && q < r_end;
+    const int c = on ? I[(size_t)q * K + slot] : -1;
+    const bool u = warp_row_used(c, slot, n, on, dummy);
+    const int key = (u && c >= c0 && c < c1) ? c : -2 - lane;  // -2 - lane matches nobody
     const unsigned peers = __match_any_sync(0xffffffffu, key);
     int pos = 0;
     if (key >= 0) {
