@@ -302,7 +302,8 @@ int llsa_attn_bwd(const llsa_desc* desc, const void* q, const void* k, const voi
   if (desc->dtype == LLSA_F32)
     return launch_status(launch_attn_bwd_simt(p, desc->dtype, (cudaStream_t)stream));
   // bf16: tensor-core kernels with TMA gathers
-  if ((((uintptr_t)dq | (uintptr_t)dk | (uintptr_t)dv) & 15) != 0) return LLSA_ERR_INVALID_ARG;
+  if ((((uintptr_t)dq | (uintptr_t)dk | (uintptr_t)dv | (uintptr_t)lse) & 15) != 0)
+    return LLSA_ERR_INVALID_ARG;  // 16-byte stores and bulk copies
   const uint64_t rows = (uint64_t)desc->B * desc->H * desc->N;
   if (rows > 0x7fffffffULL) return LLSA_ERR_UNSUPPORTED;  // TMA row coordinates are int32
   CUtensorMap maps[4];

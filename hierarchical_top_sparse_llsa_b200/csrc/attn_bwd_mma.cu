@@ -110,8 +110,9 @@ bwd_q_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
   const bool active = b < n1;
   const int K = p.K;
 
-  unsigned char* wbase = sm + (size_t)warp * TILE * 2 * kRing;
-  unsigned char* ck = sm + (size_t)kQWarps * TILE * 2 * kRing;
+  // per warp: Q | dO | kRing x (K | V) tiles
+  unsigned char* wbase = sm + (size_t)warp * TILE * (2 + 2 * kRing);
+  unsigned char* ck = sm + (size_t)kQWarps * TILE * (2 + 2 * kRing);
   unsigned char* cv = ck + (size_t)nct * TILE;
   float* clw = reinterpret_cast<float*>(cv + (size_t)nct * TILE);
   uint64_t* bars = reinterpret_cast<uint64_t*>(clw + nct * 16);
@@ -122,9 +123,10 @@ bwd_q_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
   int* flist = flist_all[warp];
 
   const uint32_t w0 = smem_u32(wbase);
+  const uint32_t qt = w0, dot = w0 + TILE;
   const uint32_t bar0 = smem_u32(bars + warp * (1 + kRing));
-  auto ring_k = [&](int st) { return w0 + (uint32_t)(2 * st) * TILE; };
-  auto ring_v = [&](int st) { return w0 + (uint32_t)(2 * st + 1) * TILE; };
+  auto ring_k = [&](int st) { return w0 + (uint32_t)(2 + 2 * st) * TILE; };
+  auto ring_v = [&](int st) { return w0 + (uint32_t)(3 + 2 * st) * TILE; };
   auto bar_of = [&](int st) { return bar0 + 8u * (1 + st); };
 
   int flags = 0;
@@ -195,20 +197,21 @@ bwd_q_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
       }
     }
   };
-  if (active && lane == 0) {
-    // Q and dO of this block land in the first ring stage before the ring starts
-    mbar_arrive_expect_tx(bar0, 2u * TILE);
-    const int y = (int)(rowbase + (size_t)b * 16);
+  if (active) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar0, 2u * TILE);
+      const int y = (int)(rowbase + (size_t)b * 16);
 #pragma unroll
-    for (int h = 0; h < HALVES; ++h) {
-      tma_load_2d(ring_k(0) + h * 2048, &tq, 64 * h, y, bar0);
-      tma_load_2d(ring_v(0) + h * 2048, &tdo, 64 * h, y, bar0);
+      for (int h = 0; h < HALVES; ++h) {
+        tma_load_2d(qt + h * 2048, &tq, 64 * h, y, bar0);
+        tma_load_2d(dot + h * 2048, &tdo, 64 * h, y, bar0);
+      }
     }
+    for (int r = 0; r < ntiles && r < kRing; ++r) issue(r);
   }
   __syncthreads();  // coarse tiles written
 
   bool ok = true;
-  uint32_t qa[D / 16][4], da[D / 16][4];
   float lse_g = 0.f, lse_g8 = 0.f, delta_g = 0.f, delta_g8 = 0.f;
   float dq[NT][4];
 #pragma unroll
@@ -217,80 +220,113 @@ bwd_q_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
   const float zero_lw[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
   if (active) {
     ok = mbar_wait_bounded(bar0, 0);
-    load_a_frags<D>(ring_k(0), lane, qa);
-    load_a_frags<D>(ring_v(0), lane, da);
     const size_t tok0 = rowbase + (size_t)b * 16 + g;
     lse_g = p.lse_in[tok0] * kLog2e;
     lse_g8 = p.lse_in[tok0 + 8] * kLog2e;
-    __syncwarp();
-    fence_proxy_async_smem();
-    for (int r = 0; r < ntiles && r < kRing; ++r) issue(r);
-
-    // sweep 1: Delta
+    // Both sweeps walk the ring tiles 0..2nf-1 with one software pipeline:
+    // S and dP of tile r+1 are issued before the elementwise work of tile r.
     float dp0 = 0.f, dp1 = 0.f;
+    float s_cur[2][4], d_cur[2][4];
     int r = 0;
-    for (; r < nf && ok; ++r) {
+    if (ntiles > 0 && ok) {
+      ok = mbar_wait_bounded(bar_of(0), 0);
+      if (ok) {
+        qk_tile_ss<D>(qt, ring_k(0), lane, s_cur);
+        qk_tile_ss<D>(dot, ring_v(0), lane, d_cur);
+      }
+    }
+    for (; r < ntiles && ok; ++r) {
       const int st = r % kRing;
-      ok = mbar_wait_bounded(bar_of(st), (uint32_t)((r / kRing) & 1));
-      if (!ok) break;
-      float s[2][4], dpv[2][4], P[2][4];
-      qk_tile<D>(qa, ring_k(st), lane, s);
-      qk_tile<D>(da, ring_v(st), lane, dpv);
-      probs_rows(s, zero_lw, sc2, lse_g, lse_g8, P);
+      float s_nx[2][4], d_nx[2][4];
+      if (r + 1 < ntiles) {
+        const int ns = (r + 1) % kRing;
+        ok = mbar_wait_bounded(bar_of(ns), (uint32_t)(((r + 1) / kRing) & 1));
+        if (!ok) break;
+        qk_tile_ss<D>(qt, ring_k(ns), lane, s_nx);
+        qk_tile_ss<D>(dot, ring_v(ns), lane, d_nx);
+      }
+      float P[2][4];
+      probs_rows(s_cur, zero_lw, sc2, lse_g, lse_g8, P);
+      if (r < nf) {  // sweep 1: Delta
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        dp0 += P[nt][0] * dpv[nt][0] + P[nt][1] * dpv[nt][1];
-        dp1 += P[nt][2] * dpv[nt][2] + P[nt][3] * dpv[nt][3];
+        for (int nt = 0; nt < 2; ++nt) {
+          dp0 += P[nt][0] * d_cur[nt][0] + P[nt][1] * d_cur[nt][1];
+          dp1 += P[nt][2] * d_cur[nt][2] + P[nt][3] * d_cur[nt][3];
+        }
+        if (r == nf - 1) {
+          // the coarse keys close sweep 1 (their tiles are resident)
+          for (int ct = 0; ct < ncpad; ++ct) {
+            float s[2][4], dpv[2][4], Pc[2][4], lw[2][2];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+              lw[nt][0] = clw[ct * 16 + 8 * nt + 2 * t];
+              lw[nt][1] = clw[ct * 16 + 8 * nt + 2 * t + 1];
+            }
+            qk_tile_ss<D>(qt, smem_u32(ck) + ct * TILE, lane, s);
+            qk_tile_ss<D>(dot, smem_u32(cv) + ct * TILE, lane, dpv);
+            probs_rows(s, lw, sc2, lse_g, lse_g8, Pc);
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+              dp0 += Pc[nt][0] * dpv[nt][0] + Pc[nt][1] * dpv[nt][1];
+              dp1 += Pc[nt][2] * dpv[nt][2] + Pc[nt][3] * dpv[nt][3];
+            }
+          }
+          dp0 += __shfl_xor_sync(0xffffffffu, dp0, 1);
+          dp0 += __shfl_xor_sync(0xffffffffu, dp0, 2);
+          dp1 += __shfl_xor_sync(0xffffffffu, dp1, 1);
+          dp1 += __shfl_xor_sync(0xffffffffu, dp1, 2);
+          delta_g = dp0;
+          delta_g8 = dp1;
+        }
+      } else {  // sweep 2: dQ += dS K
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) P[nt][e] *= d_cur[nt][e] - ((e < 2) ? delta_g : delta_g8);
+        uint32_t dsa[4];
+        pack_frag(P, dsa);
+        pv_tile<D>(dsa, ring_k(st), lane, dq);
       }
       __syncwarp();
       fence_proxy_async_smem();
       if (r + kRing < ntiles) issue(r + kRing);
-    }
-    for (int ct = 0; ct < ncpad && ok; ++ct) {
-      float s[2][4], dpv[2][4], P[2][4], lw[2][2];
+      if (r + 1 < ntiles) {
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        lw[nt][0] = clw[ct * 16 + 8 * nt + 2 * t];
-        lw[nt][1] = clw[ct * 16 + 8 * nt + 2 * t + 1];
-      }
-      qk_tile<D>(qa, smem_u32(ck) + ct * TILE, lane, s);
-      qk_tile<D>(da, smem_u32(cv) + ct * TILE, lane, dpv);
-      probs_rows(s, lw, sc2, lse_g, lse_g8, P);
+        for (int a2 = 0; a2 < 2; ++a2)
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        dp0 += P[nt][0] * dpv[nt][0] + P[nt][1] * dpv[nt][1];
-        dp1 += P[nt][2] * dpv[nt][2] + P[nt][3] * dpv[nt][3];
+          for (int e = 0; e < 4; ++e) {
+            s_cur[a2][e] = s_nx[a2][e];
+            d_cur[a2][e] = d_nx[a2][e];
+          }
       }
     }
-    dp0 += __shfl_xor_sync(0xffffffffu, dp0, 1);
-    dp0 += __shfl_xor_sync(0xffffffffu, dp0, 2);
-    dp1 += __shfl_xor_sync(0xffffffffu, dp1, 1);
-    dp1 += __shfl_xor_sync(0xffffffffu, dp1, 2);
-    delta_g = dp0;
-    delta_g8 = dp1;
+    if (nf == 0 && ok) {  // no fine keys: Delta from the coarse keys alone
+      for (int ct = 0; ct < ncpad; ++ct) {
+        float s[2][4], dpv[2][4], Pc[2][4], lw[2][2];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          lw[nt][0] = clw[ct * 16 + 8 * nt + 2 * t];
+          lw[nt][1] = clw[ct * 16 + 8 * nt + 2 * t + 1];
+        }
+        qk_tile_ss<D>(qt, smem_u32(ck) + ct * TILE, lane, s);
+        qk_tile_ss<D>(dot, smem_u32(cv) + ct * TILE, lane, dpv);
+        probs_rows(s, lw, sc2, lse_g, lse_g8, Pc);
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          dp0 += Pc[nt][0] * dpv[nt][0] + Pc[nt][1] * dpv[nt][1];
+          dp1 += Pc[nt][2] * dpv[nt][2] + Pc[nt][3] * dpv[nt][3];
+        }
+      }
+      dp0 += __shfl_xor_sync(0xffffffffu, dp0, 1);
+      dp0 += __shfl_xor_sync(0xffffffffu, dp0, 2);
+      dp1 += __shfl_xor_sync(0xffffffffu, dp1, 1);
+      dp1 += __shfl_xor_sync(0xffffffffu, dp1, 2);
+      delta_g = dp0;
+      delta_g8 = dp1;
+    }
     if (t == 0) {
       p.delta[tok0] = delta_g;
       p.delta[tok0 + 8] = delta_g8;
-    }
-    // sweep 2: dQ from the fine keys
-    for (; r < ntiles && ok; ++r) {
-      const int st = r % kRing;
-      ok = mbar_wait_bounded(bar_of(st), (uint32_t)((r / kRing) & 1));
-      if (!ok) break;
-      float s[2][4], dpv[2][4], P[2][4];
-      qk_tile<D>(qa, ring_k(st), lane, s);
-      qk_tile<D>(da, ring_v(st), lane, dpv);
-      probs_rows(s, zero_lw, sc2, lse_g, lse_g8, P);
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) P[nt][e] *= dpv[nt][e] - ((e < 2) ? delta_g : delta_g8);
-      uint32_t dsa[4];
-      pack_frag(P, dsa);
-      pv_tile<D>(dsa, ring_k(st), lane, dq);
-      __syncwarp();
-      fence_proxy_async_smem();
-      if (r + kRing < ntiles) issue(r + kRing);
     }
     if (!ok) {
       for (int q = r; q < ntiles && q < r + kRing; ++q)
@@ -301,7 +337,7 @@ bwd_q_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
 
   // coarse keys: dQ share and the per-CTA partials, reduced in warp order
   const int NG = n1 / kQWarps;
-  float* stage = reinterpret_cast<float*>(wbase);  // [2][16][D] fp32, reuses this warp's ring
+  float* stage = reinterpret_cast<float*>(wbase + 2 * TILE);  // [2][16][D] fp32, reuses this warp's ring
   for (int ct = 0; ct < ncpad; ++ct) {
     if (active && ok) {
       float s[2][4], dpv[2][4], P[2][4], dS[2][4], lw[2][2];
@@ -310,13 +346,16 @@ bwd_q_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
         lw[nt][0] = clw[ct * 16 + 8 * nt + 2 * t];
         lw[nt][1] = clw[ct * 16 + 8 * nt + 2 * t + 1];
       }
-      qk_tile<D>(qa, smem_u32(ck) + ct * TILE, lane, s);
-      qk_tile<D>(da, smem_u32(cv) + ct * TILE, lane, dpv);
+      qk_tile_ss<D>(qt, smem_u32(ck) + ct * TILE, lane, s);
+      qk_tile_ss<D>(dot, smem_u32(cv) + ct * TILE, lane, dpv);
       probs_rows(s, lw, sc2, lse_g, lse_g8, P);
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) dS[nt][e] = P[nt][e] * (dpv[nt][e] - ((e < 2) ? delta_g : delta_g8));
+      uint32_t qa[D / 16][4], da[D / 16][4];
+      load_a_frags<D>(qt, lane, qa);
+      load_a_frags<D>(dot, lane, da);
       uint32_t dsh[4], dsl[4], ph[4], pl[4], dsth[4], dstl[4], pth[4], ptl[4];
       split_frag(dS, dsh, dsl);
       split_frag(P, ph, pl);
@@ -361,7 +400,7 @@ bwd_q_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
       if (ck_idx >= nc) continue;
       float a = 0.f;
       for (int w = 0; w < kQWarps; ++w)
-        a += reinterpret_cast<const float*>(sm + (size_t)w * TILE * 2 * kRing)[e];
+        a += reinterpret_cast<const float*>(sm + (size_t)w * TILE * (2 + 2 * kRing) + 2 * TILE)[e];
       const int l = clist[ck_idx] >> 24;
       float* part = p.part[l] + ((((size_t)bh * NG + grp) * K + cslot[ck_idx]) * 2 + kv) * D + d;
       *part = (kv == 0) ? a * p.scale : a;
@@ -392,6 +431,10 @@ bwd_kv_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
   constexpr int TILE = 32 * D;
   constexpr int NT = D / 8;
   constexpr int HALVES = D / 64;
+  constexpr int SIDE = 128;  // LSE[16] and Delta[16] of a stage's query block (fp32)
+  // per warp: K_c | V_c | kRing x (Q | dO) tiles, then kRing side buffers; every
+  // tile stays 1024-byte aligned for the 128-byte swizzle
+  constexpr int WARP_BYTES = 2 * TILE * (1 + kRing) + 1024;
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -404,10 +447,15 @@ bwd_kv_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
   const bool active = c < n1;
   const int K = p.K;
 
-  const uint32_t w0 = smem_u32(sm + (size_t)warp * TILE * (2 + 2 * kRing));
+  unsigned char* wb = sm + (size_t)warp * WARP_BYTES;
+  const uint32_t w0 = smem_u32(wb);
   const uint32_t kt = w0, vt = w0 + TILE;
   auto ring_q = [&](int st) { return w0 + (uint32_t)(2 + 2 * st) * TILE; };
   auto ring_do = [&](int st) { return w0 + (uint32_t)(3 + 2 * st) * TILE; };
+  const uint32_t side0 = w0 + (uint32_t)(2 + 2 * kRing) * TILE;
+  auto side_of = [&](int st) {
+    return reinterpret_cast<const float*>(wb + (2 + 2 * kRing) * TILE + st * SIDE);
+  };
   const uint32_t bar0 = smem_u32(&bars_all[warp][0]);
   auto bar_of = [&](int st) { return bar0 + 8u * (1 + st); };
   if (lane == 0) {
@@ -426,13 +474,16 @@ bwd_kv_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
     if (lane == 0) {
       const int qb = col[beg + r];
       const int st = r % kRing;
-      mbar_arrive_expect_tx(bar_of(st), 2u * TILE);
-      const int y = (int)(rowbase + (size_t)qb * 16);
+      mbar_arrive_expect_tx(bar_of(st), 2u * TILE + SIDE);
+      const size_t row0 = rowbase + (size_t)qb * 16;
+      const int y = (int)row0;
 #pragma unroll
       for (int h = 0; h < HALVES; ++h) {
         tma_load_2d(ring_q(st) + h * 2048, &tq, 64 * h, y, bar_of(st));
         tma_load_2d(ring_do(st) + h * 2048, &tdo, 64 * h, y, bar_of(st));
       }
+      bulk_load(side0 + st * SIDE, p.lse_in + row0, 64, bar_of(st));
+      bulk_load(side0 + st * SIDE + 64, p.delta + row0, 64, bar_of(st));
     }
   };
   if (lane == 0) {
@@ -447,9 +498,6 @@ bwd_kv_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
   for (int r = 0; r < nq && r < kRing; ++r) issue(r);
 
   bool ok = mbar_wait_bounded(bar0, 0);
-  uint32_t ka[D / 16][4], va[D / 16][4];
-  load_a_frags<D>(kt, lane, ka);
-  load_a_frags<D>(vt, lane, va);
   float dk[NT][4], dv[NT][4];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) {
@@ -457,32 +505,38 @@ bwd_kv_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
     dv[nt][0] = dv[nt][1] = dv[nt][2] = dv[nt][3] = 0.f;
   }
   const float sc2 = p.scale * kLog2e;
+  // software pipeline: S^T and dP^T of query block r+1 are issued before the
+  // elementwise step and the dV/dK products of block r
+  float s_cur[2][4], d_cur[2][4];
   int r = 0;
+  if (nq > 0 && ok) {
+    ok = mbar_wait_bounded(bar_of(0), 0);
+    if (ok) {
+      qk_tile_ss<D>(kt, ring_q(0), lane, s_cur);
+      qk_tile_ss<D>(vt, ring_do(0), lane, d_cur);
+    }
+  }
   for (; r < nq && ok; ++r) {
     const int st = r % kRing;
-    const int qb = col[beg + r];
+    float s_nx[2][4], d_nx[2][4];
+    if (r + 1 < nq) {
+      const int ns = (r + 1) % kRing;
+      ok = mbar_wait_bounded(bar_of(ns), (uint32_t)(((r + 1) / kRing) & 1));
+      if (!ok) break;
+      qk_tile_ss<D>(kt, ring_q(ns), lane, s_nx);
+      qk_tile_ss<D>(vt, ring_do(ns), lane, d_nx);
+    }
     // LSE and Delta of the queries in this thread's columns: 2t, 2t+1, 8+2t, 9+2t
-    const size_t q0 = rowbase + (size_t)qb * 16;
-    float lse[2][2], dl[2][2];
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        lse[nt][e] = p.lse_in[q0 + 8 * nt + 2 * t + e] * kLog2e;
-        dl[nt][e] = p.delta[q0 + 8 * nt + 2 * t + e];
-      }
-    ok = mbar_wait_bounded(bar_of(st), (uint32_t)((r / kRing) & 1));
-    if (!ok) break;
-    float s[2][4], dpv[2][4], P[2][4], dS[2][4];
-    qk_tile<D>(ka, ring_q(st), lane, s);    // S^T: rows keys, columns queries
-    qk_tile<D>(va, ring_do(st), lane, dpv); // dP^T
+    const float* side = side_of(st);
+    float P[2][4], dS[2][4];
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float l2 = lse[nt][e & 1];
-        P[nt][e] = (l2 == -INFINITY) ? 0.f : exp2f(fmaf(s[nt][e], sc2, -l2));
-        dS[nt][e] = P[nt][e] * (dpv[nt][e] - dl[nt][e & 1]);
+        const int qi = 8 * nt + 2 * t + (e & 1);
+        const float l2 = side[qi] * kLog2e;
+        P[nt][e] = (l2 == -INFINITY) ? 0.f : exp2f(fmaf(s_cur[nt][e], sc2, -l2));
+        dS[nt][e] = P[nt][e] * (d_cur[nt][e] - side[16 + qi]);
       }
     uint32_t ph[4], pl[4], dsh[4], dsl[4];
     split_frag(P, ph, pl);
@@ -492,6 +546,15 @@ bwd_kv_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
     __syncwarp();
     fence_proxy_async_smem();
     if (r + kRing < nq) issue(r + kRing);
+    if (r + 1 < nq) {
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          s_cur[a][e] = s_nx[a][e];
+          d_cur[a][e] = d_nx[a][e];
+        }
+    }
   }
   if (!ok) {
     for (int q = r; q < nq && q < r + kRing; ++q)
@@ -533,7 +596,7 @@ cudaError_t launch_typed(const AttnParams& p, const CUtensorMap* maps, cudaStrea
   const int n1 = p.N / kBlock;
   const int nct = ((p.L - 1) * p.K + 15) / 16;
   // pass 1
-  const size_t smem1 = 1024 + (size_t)kQWarps * TILE * 2 * kRing + 2 * (size_t)nct * TILE +
+  const size_t smem1 = 1024 + (size_t)kQWarps * TILE * (2 + 2 * kRing) + 2 * (size_t)nct * TILE +
                        nct * 16 * sizeof(float) + kQWarps * (1 + kRing) * 8 + 2 * nct * 16 * sizeof(int);
   cudaError_t e = cudaFuncSetAttribute(bwd_q_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
   if (e != cudaSuccess) return e;
@@ -545,7 +608,7 @@ cudaError_t launch_typed(const AttnParams& p, const CUtensorMap* maps, cudaStrea
   e = launch_coarse_reduce(p, s);
   if (e != cudaSuccess) return e;
   // pass 3
-  const size_t smem3 = 1024 + (size_t)kKVWarps * TILE * (2 + 2 * kRing);
+  const size_t smem3 = 1024 + (size_t)kKVWarps * (2 * TILE * (1 + kRing) + 1024);
   e = cudaFuncSetAttribute(bwd_kv_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3);
   if (e != cudaSuccess) return e;
   bwd_kv_mma_kernel<D><<<dim3((n1 + kKVWarps - 1) / kKVWarps, BH), kKVWarps * 32, smem3, s>>>(

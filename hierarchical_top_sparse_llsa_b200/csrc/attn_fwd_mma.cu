@@ -3,16 +3,17 @@
 // of "Trainable Log-linear Sparse Attention for Efficient Diffusion
 // Transformers").
 //
-// One warp owns one 16-token query block (the block is exactly the M = 16 of
-// the warp MMA).  Its selected 16-token key blocks are contiguous 16-row
-// tiles of K and V, gathered by 2D TMA loads (128-byte swizzle, no
-// multicast) into a 2-stage ring with one mbarrier per stage (the Q tile
-// passes through stage 0 first); S of the next tile is issued before the
-// softmax and PV of the current one, so the MMA pipe has work while the
-// exponentials run.  A CTA holds 4
-// sibling query blocks (same level-2 ancestor), which share every coarse
-// key; the coarse K/V rows (fp32 pyramid) are converted once per CTA to bf16
-// tiles in shared memory, with ln(w_l) per key folded into the scores.
+// One warp owns 4 consecutive 16-token query blocks, one after the other (a
+// block is exactly the M = 16 of the warp MMA); a CTA of 4 warps covers the
+// 16 blocks under one level-2 token, which share every coarse key.  The
+// selected 16-token key blocks of a warp's 4 blocks form one stream of
+// contiguous 16-row K/V tiles, gathered by 2D TMA loads (128-byte swizzle, no
+// multicast) into a 2-stage ring that runs on across block boundaries, and
+// the next block's Q tile is loaded into a second buffer while the current
+// block is computed, so set-up latency is paid once per warp, not per block.
+// S of the next tile is issued before the softmax and PV of the current one.
+// The coarse K/V rows (fp32 pyramid) are converted once per CTA to bf16 tiles
+// in shared memory, with ln(w_l) per key folded into the scores.
 // S = Q K^T and O += P V run on m16n8k16 bf16 MMAs with fp32 accumulation;
 // the softmax is online, in base 2, in fp32 registers.
 
@@ -25,7 +26,8 @@ namespace llsa {
 
 namespace {
 
-constexpr int kFwdWarps = 4;
+constexpr int kFwdWarps = 4;  // warps per CTA
+constexpr int kBPW = 4;       // consecutive query blocks per warp (same coarse keys)
 constexpr int kStages = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -101,40 +103,53 @@ attn_fwd_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
   const int g = lane >> 2, t = lane & 3;
   const int bh = blockIdx.y;
   const int n1 = p.N >> 4;
-  const int b = blockIdx.x * kFwdWarps + warp;
-  const bool active = b < n1;
+  const int wb0 = (blockIdx.x * kFwdWarps + warp) * kBPW;  // this warp's first block
   const int K = p.K;
 
-  unsigned char* wbase = sm + (size_t)warp * TILE * 2 * kStages;
-  unsigned char* ck = sm + (size_t)kFwdWarps * TILE * 2 * kStages;
+  // per warp: 2 Q buffers | kStages x (K | V); then coarse K, coarse V, ...
+  unsigned char* wbase = sm + (size_t)warp * TILE * (2 + 2 * kStages);
+  unsigned char* ck = sm + (size_t)kFwdWarps * TILE * (2 + 2 * kStages);
   unsigned char* cv = ck + (size_t)nct * TILE;
   float* clw = reinterpret_cast<float*>(cv + (size_t)nct * TILE);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(clw + nct * 16);
-  int* clist = reinterpret_cast<int*>(bars + kFwdWarps * (kStages + 1));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(clw + nct * 16);  // per warp: 2 Q, kStages ring
+  int* clist = reinterpret_cast<int*>(bars + kFwdWarps * (2 + kStages));
   __shared__ int s_nc;
-  __shared__ int flist_all[kFwdWarps][32];  // each warp's used fine blocks, ascending
-  int* flist = flist_all[warp];
+  __shared__ int flist_all[kFwdWarps][kBPW][32];  // used fine blocks of each block, ascending
+  __shared__ int foff_all[kFwdWarps][kBPW + 1];   // stream offset of each block's tiles
 
   const uint32_t w0 = smem_u32(wbase);
-  const uint32_t bar0 = smem_u32(bars + warp * (kStages + 1));  // [0] = Q, [1..] = stages
-  auto stage_k = [&](int st) { return w0 + (uint32_t)(2 * st) * TILE; };
-  auto stage_v = [&](int st) { return w0 + (uint32_t)(2 * st + 1) * TILE; };
-  auto bar_of = [&](int st) { return bar0 + 8u * (1 + st); };
+  auto qbuf = [&](int i) { return w0 + (uint32_t)(i & 1) * TILE; };
+  auto stage_k = [&](int st) { return w0 + (uint32_t)(2 + 2 * st) * TILE; };
+  auto stage_v = [&](int st) { return w0 + (uint32_t)(3 + 2 * st) * TILE; };
+  const uint32_t bar0 = smem_u32(bars + warp * (2 + kStages));
+  auto qbar = [&](int i) { return bar0 + 8u * (i & 1); };
+  auto bar_of = [&](int st) { return bar0 + 8u * (2 + st); };
 
   int flags = 0;
-  // ---- this warp's fine blocks (lane s holds slot s of its row of I(1))
-  const bool on_row = active && lane < K;
-  const int my_blk = on_row ? p.idx[1][((size_t)bh * n1 + b) * K + lane] : -1;
-  const bool used = warp_row_used(my_blk, lane, n1, on_row, flags);
-  const unsigned fmask = __ballot_sync(0xffffffffu, used);
-  const int nf = __popc(fmask);
-  if (used) flist[__popc(fmask & ((1u << lane) - 1u))] = my_blk;
-  __syncwarp();
-
+  // ---- fine lists of this warp's blocks
+  int (*flist)[32] = flist_all[warp];
+  int* foff = foff_all[warp];
+  int nblk = 0;  // active blocks of this warp
+  {
+    int off = 0;
+#pragma unroll
+    for (int i = 0; i < kBPW; ++i) {
+      const int b = wb0 + i;
+      const bool on = (b < n1) && lane < K;
+      const int v = on ? p.idx[1][((size_t)bh * n1 + b) * K + lane] : -1;
+      const bool used = warp_row_used(v, lane, n1, on, flags);
+      const unsigned m = __ballot_sync(0xffffffffu, used);
+      if (used) flist[i][__popc(m & ((1u << lane) - 1u))] = v;
+      if (lane == 0) foff[i] = off;
+      off += __popc(m);
+      if (b < n1) nblk = i + 1;
+    }
+    if (lane == 0) foff[kBPW] = off;
+  }
   // ---- coarse keys shared by the CTA (warp 0 builds the list)
   if (warp == 0) {
     int n = 0;
-    const int b0 = blockIdx.x * kFwdWarps;
+    const int b0 = blockIdx.x * kFwdWarps * kBPW;
     for (int l = 2; l <= p.L; ++l) {
       const int nl = p.N >> (4 * l);
       const int a = b0 >> (4 * (l - 1));
@@ -147,10 +162,40 @@ attn_fwd_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
     if (lane == 0) s_nc = n;
   }
   if (lane == 0) {
-    for (int i = 0; i <= kStages; ++i) mbar_init(bar0 + 8u * i, 1);
+    for (int i = 0; i < 2 + kStages; ++i) mbar_init(bar0 + 8u * i, 1);
     fence_mbar_init();
   }
-  __syncthreads();
+  __syncwarp();
+  const size_t rowbase = (size_t)bh * p.N;
+  const int T = foff[kBPW];  // tiles in this warp's stream
+  // stream item j -> (block, fine index)
+  auto issue_item = [&](int j) {
+    if (lane == 0) {
+      int i = 0;
+      while (j >= foff[i + 1]) ++i;
+      const int blk = flist[i][j - foff[i]];
+      const int st = j % kStages;
+      mbar_arrive_expect_tx(bar_of(st), 2u * TILE);
+      const int y = (int)(rowbase + (size_t)blk * 16);
+#pragma unroll
+      for (int h = 0; h < HALVES; ++h) {
+        tma_load_2d(stage_k(st) + h * 2048, &tk, 64 * h, y, bar_of(st));
+        tma_load_2d(stage_v(st) + h * 2048, &tv, 64 * h, y, bar_of(st));
+      }
+    }
+  };
+  auto issue_q = [&](int i) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(qbar(i), TILE);
+      const int y = (int)(rowbase + (size_t)(wb0 + i) * 16);
+#pragma unroll
+      for (int h = 0; h < HALVES; ++h) tma_load_2d(qbuf(i) + h * 2048, &tq, 64 * h, y, qbar(i));
+    }
+  };
+  for (int i = 0; i < nblk && i < 2; ++i) issue_q(i);
+  for (int j = 0; j < T && j < kStages; ++j) issue_item(j);
+
+  __syncthreads();  // coarse list and every warp's barriers ready
   const int nc = s_nc;
   const int ncpad = (nc + 15) >> 4;
   // coarse rows: fp32 pyramid -> bf16 swizzled tiles; padded keys are zero
@@ -173,118 +218,96 @@ attn_fwd_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
   }
   for (int e = threadIdx.x; e < ncpad * 16; e += blockDim.x)
     clw[e] = (e < nc) ? p.logw[clist[e] >> 24] * kLog2e : -INFINITY;
-
-  // ---- Q lands in stage 0 first; the fine tiles follow once its fragments are read
-  const size_t rowbase = (size_t)bh * p.N;
-  auto issue_block = [&](int r) {
-    if (lane == 0) {
-      const int blk = flist[r];
-      const int st = r % kStages;
-      mbar_arrive_expect_tx(bar_of(st), 2u * TILE);
-      const int y = (int)(rowbase + (size_t)blk * 16);
-#pragma unroll
-      for (int h = 0; h < HALVES; ++h) {
-        tma_load_2d(stage_k(st) + h * 2048, &tk, 64 * h, y, bar_of(st));
-        tma_load_2d(stage_v(st) + h * 2048, &tv, 64 * h, y, bar_of(st));
-      }
-    }
-  };
-  if (active) {
-    if (lane == 0) {
-      mbar_arrive_expect_tx(bar0, TILE);
-#pragma unroll
-      for (int h = 0; h < HALVES; ++h)
-        tma_load_2d(stage_k(0) + h * 2048, &tq, 64 * h, (int)(rowbase + (size_t)b * 16), bar0);
-    }
-    if (nf > 1) issue_block(1);  // stage 1 is free; stage 0 holds Q for now
-  }
   __syncthreads();  // coarse tiles written
-  if (!active) return;
 
-  bool ok = mbar_wait_bounded(bar0, 0);
-  uint32_t qa[D / 16][4];
-  load_a_frags<D>(stage_k(0), lane, qa);
-  __syncwarp();
-  fence_proxy_async_smem();
-  if (nf > 0) issue_block(0);
-
-  float o[NT][4];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
-  SoftmaxState st;
-  st.m[0] = st.m[1] = -INFINITY;
-  st.l[0] = st.l[1] = 0.f;
   const float sc2 = p.scale * kLog2e;
   const float zero_lw[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-
-  // software pipeline: S of tile r+1 is issued before the softmax and PV of tile r
-  float s_cur[2][4];
-  int r = 0;
-  if (nf > 0 && ok) {
-    ok = mbar_wait_bounded(bar_of(0), 0);
-    if (ok) qk_tile<D>(qa, stage_k(0), lane, s_cur);
-  }
-  for (; r < nf && ok; ++r) {
-    const int sidx = r % kStages;
-    float s_next[2][4];
-    if (r + 1 < nf) {
-      const int nidx = (r + 1) % kStages;
-      ok = mbar_wait_bounded(bar_of(nidx), (uint32_t)(((r + 1) / kStages) & 1));
-      if (!ok) break;
-      qk_tile<D>(qa, stage_k(nidx), lane, s_next);
-    }
-    uint32_t pa[4];
-    softmax_tile<NT>(s_cur, zero_lw, sc2, st, o, pa);
-    pv_tile<D>(pa, stage_v(sidx), lane, o);
+  bool ok = true;
+  int j = 0;  // next stream item
+  for (int i = 0; i < nblk && ok; ++i) {
+    const int b = wb0 + i;
+    ok = mbar_wait_bounded(qbar(i), (uint32_t)((i >> 1) & 1));
+    if (!ok) break;
+    uint32_t qa[D / 16][4];
+    load_a_frags<D>(qbuf(i), lane, qa);
     __syncwarp();
     fence_proxy_async_smem();
-    if (r + kStages < nf) issue_block(r + kStages);
-    if (r + 1 < nf) {
+    if (i + 2 < nblk) issue_q(i + 2);  // this Q buffer is free again
+
+    float o[NT][4];
 #pragma unroll
-      for (int a = 0; a < 2; ++a)
+    for (int nt = 0; nt < NT; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
+    SoftmaxState st;
+    st.m[0] = st.m[1] = -INFINITY;
+    st.l[0] = st.l[1] = 0.f;
+    const int jend = foff[i + 1];
+    float s_cur[2][4];
+    if (j < jend) {
+      ok = mbar_wait_bounded(bar_of(j % kStages), (uint32_t)((j / kStages) & 1));
+      if (!ok) break;
+      qk_tile<D>(qa, stage_k(j % kStages), lane, s_cur);
+    }
+    for (; j < jend; ++j) {
+      const int sidx = j % kStages;
+      float s_nx[2][4];
+      if (j + 1 < jend) {
+        const int nidx = (j + 1) % kStages;
+        ok = mbar_wait_bounded(bar_of(nidx), (uint32_t)(((j + 1) / kStages) & 1));
+        if (!ok) break;
+        qk_tile<D>(qa, stage_k(nidx), lane, s_nx);
+      }
+      uint32_t pa[4];
+      softmax_tile<NT>(s_cur, zero_lw, sc2, st, o, pa);
+      pv_tile<D>(pa, stage_v(sidx), lane, o);
+      __syncwarp();
+      fence_proxy_async_smem();
+      if (j + kStages < T) issue_item(j + kStages);
+      if (j + 1 < jend) {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) s_cur[a][e] = s_next[a][e];
+        for (int a2 = 0; a2 < 2; ++a2)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) s_cur[a2][e] = s_nx[a2][e];
+      }
+    }
+    if (!ok) break;
+    for (int ct = 0; ct < ncpad; ++ct) {
+      float s[2][4];
+      uint32_t pa[4];
+      qk_tile<D>(qa, smem_u32(ck) + ct * TILE, lane, s);
+      float lw[2][2];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        lw[nt][0] = clw[ct * 16 + 8 * nt + 2 * t];
+        lw[nt][1] = clw[ct * 16 + 8 * nt + 2 * t + 1];
+      }
+      softmax_tile<NT>(s, lw, sc2, st, o, pa);
+      pv_tile<D>(pa, smem_u32(cv) + ct * TILE, lane, o);
+    }
+    // ---- epilogue: O = acc / l, LSE = ln(sum) = (m + log2 l) ln 2
+    float l0 = st.l[0], l1 = st.l[1];
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    const float i0 = l0 > 0.f ? 1.f / l0 : 0.f;
+    const float i1 = l1 > 0.f ? 1.f / l1 : 0.f;
+    bf16* O = static_cast<bf16*>(p.out);
+    const size_t tok0 = rowbase + (size_t)b * 16 + g;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      *reinterpret_cast<uint32_t*>(O + tok0 * D + 8 * nt + 2 * t) = pack_bf16(o[nt][0] * i0, o[nt][1] * i0);
+      *reinterpret_cast<uint32_t*>(O + (tok0 + 8) * D + 8 * nt + 2 * t) = pack_bf16(o[nt][2] * i1, o[nt][3] * i1);
+    }
+    if (t == 0) {
+      p.lse[tok0] = l0 > 0.f ? (st.m[0] + log2f(l0)) * kLn2 : -INFINITY;
+      p.lse[tok0 + 8] = l1 > 0.f ? (st.m[1] + log2f(l1)) * kLn2 : -INFINITY;
     }
   }
   if (!ok) {
     // give the copies already in flight a bounded chance to land, then stop
-    for (int q = r; q < nf && q < r + kStages; ++q)
+    for (int q = j; q < T && q < j + kStages; ++q)
       mbar_wait_bounded(bar_of(q % kStages), (uint32_t)((q / kStages) & 1));
-    if (lane == 0) report_status(p.status, LLSA_DEV_TIMEOUT);
-    return;
-  }
-  for (int ct = 0; ct < ncpad; ++ct) {
-    float s[2][4];
-    uint32_t pa[4];
-    qk_tile<D>(qa, smem_u32(ck) + ct * TILE, lane, s);
-    float lw[2][2];
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      lw[nt][0] = clw[ct * 16 + 8 * nt + 2 * t];
-      lw[nt][1] = clw[ct * 16 + 8 * nt + 2 * t + 1];
-    }
-    softmax_tile<NT>(s, lw, sc2, st, o, pa);
-    pv_tile<D>(pa, smem_u32(cv) + ct * TILE, lane, o);
-  }
-
-  // ---- epilogue: O = acc / l, LSE = ln(sum) = (m + log2 l) ln 2
-  float l0 = st.l[0], l1 = st.l[1];
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-  l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-  l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-  const float i0 = l0 > 0.f ? 1.f / l0 : 0.f;
-  const float i1 = l1 > 0.f ? 1.f / l1 : 0.f;
-  bf16* O = static_cast<bf16*>(p.out);
-  const size_t tok0 = rowbase + (size_t)b * 16 + g;
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    *reinterpret_cast<uint32_t*>(O + tok0 * D + 8 * nt + 2 * t) = pack_bf16(o[nt][0] * i0, o[nt][1] * i0);
-    *reinterpret_cast<uint32_t*>(O + (tok0 + 8) * D + 8 * nt + 2 * t) = pack_bf16(o[nt][2] * i1, o[nt][3] * i1);
-  }
-  if (t == 0) {
-    p.lse[tok0] = l0 > 0.f ? (st.m[0] + log2f(l0)) * kLn2 : -INFINITY;
-    p.lse[tok0 + 8] = l1 > 0.f ? (st.m[1] + log2f(l1)) * kLn2 : -INFINITY;
+    flags |= LLSA_DEV_TIMEOUT;
   }
   flags = __reduce_or_sync(0xffffffffu, flags);
   if (lane == 0) report_status(p.status, flags);
@@ -294,13 +317,14 @@ template <int D>
 cudaError_t launch_typed(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s) {
   constexpr int TILE = 32 * D;
   const int nct = ((p.L - 1) * p.K + 15) / 16;
-  const size_t smem = 1024 + (size_t)kFwdWarps * TILE * 2 * kStages + 2 * (size_t)nct * TILE +
-                      nct * 16 * sizeof(float) + kFwdWarps * (kStages + 1) * 8 + nct * 16 * sizeof(int);
+  const size_t smem = 1024 + (size_t)kFwdWarps * TILE * (2 + 2 * kStages) + 2 * (size_t)nct * TILE +
+                      nct * 16 * sizeof(float) + kFwdWarps * (2 + kStages) * 8 + nct * 16 * sizeof(int);
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_mma_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int n1 = p.N / kBlock;
-  dim3 grid((n1 + kFwdWarps - 1) / kFwdWarps, p.B * p.H);
+  const int per_cta = kFwdWarps * kBPW;
+  dim3 grid((n1 + per_cta - 1) / per_cta, p.B * p.H);
   attn_fwd_mma_kernel<D><<<grid, kFwdWarps * 32, smem, s>>>(maps[0], maps[1], maps[2], p, nct);
   return cudaGetLastError();
 }

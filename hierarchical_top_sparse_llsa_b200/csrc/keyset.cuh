@@ -64,3 +64,79 @@ __device__ __forceinline__ int build_key_list(KeyList& kl, const AttnParams& p, 
 }
 
 }  // namespace llsa
+
+namespace llsa {
+
+// Ascending bitonic sort of 32*E ints held by one warp, element i = lane + 32*e
+// in v[e] (E a power of two).  All 32 lanes must call it.
+template <int E>
+__device__ __forceinline__ void warp_bitonic_sort(int (&v)[E], int lane) {
+  constexpr int n = 32 * E;
+#pragma unroll
+  for (int k = 2; k <= n; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j < 32) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const int i = lane + 32 * e;
+          const int other = __shfl_xor_sync(0xffffffffu, v[e], j);
+          const bool lower = (lane & j) == 0;
+          const bool asc = (i & k) == 0;
+          v[e] = (asc == lower) ? min(v[e], other) : max(v[e], other);
+        }
+      } else {
+        const int je = j / 32;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          if ((e & je) == 0) {
+            const int i = lane + 32 * e;
+            const bool asc = (i & k) == 0;
+            const int a = v[e], b = v[e + je];
+            v[e] = asc ? min(a, b) : max(a, b);
+            v[e + je] = asc ? max(a, b) : min(a, b);
+          }
+        }
+      }
+    }
+  }
+}
+
+// Sorted, de-duplicated union of `cnt` entries in[0..cnt) (cnt <= 32*E) into
+// out[0..u); returns u.  One warp; entries >= 0x7fffffff are ignored.
+template <int E>
+__device__ __forceinline__ int warp_sorted_union(const int* in, int cnt, int* out, int lane) {
+  int v[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int i = lane + 32 * e;
+    v[e] = (i < cnt) ? in[i] : 0x7fffffff;
+  }
+  warp_bitonic_sort<E>(v, lane);
+  int base = 0;
+  int prev_last = -1;  // last element of the previous column (e - 1), lane 31
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    int prev = __shfl_up_sync(0xffffffffu, v[e], 1);
+    if (lane == 0) prev = prev_last;
+    const bool first = v[e] != 0x7fffffff && v[e] != prev;
+    const unsigned m = __ballot_sync(0xffffffffu, first);
+    if (first) out[base + __popc(m & ((1u << lane) - 1u))] = v[e];
+    base += __popc(m);
+    prev_last = __shfl_sync(0xffffffffu, v[e], 31);
+  }
+  return base;
+}
+
+// Position of `x` in the sorted array a[0..n) (x must be present).
+__device__ __forceinline__ int sorted_find(const int* a, int n, int x) {
+  int lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (a[mid] < x) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo;
+}
+
+}  // namespace llsa

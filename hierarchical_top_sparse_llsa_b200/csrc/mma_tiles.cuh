@@ -38,6 +38,29 @@ __device__ __forceinline__ void qk_tile(const uint32_t (&qa)[D / 16][4], uint32_
   }
 }
 
+// The same with the A operand read from a 16-row tile `at` in shared memory
+// (fragments loaded per k-step instead of held in registers).
+template <int D>
+__device__ __forceinline__ void qk_tile_ss(uint32_t at, uint32_t kt, int lane, float (&s)[2][4]) {
+  const int mi = lane >> 3;
+  const int arow = (mi & 1) * 8 + (lane & 7);
+  const int ac = mi >> 1;
+  const int krow = (mi >> 1) * 8 + (lane & 7);
+  const int kc = mi & 1;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) s[nt][e] = 0.f;
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    uint32_t a[4], b0, b1, b2, b3;
+    ldsm_x4(at + swz(arow, 2 * kk + ac), a[0], a[1], a[2], a[3]);
+    ldsm_x4(kt + swz(krow, 2 * kk + kc), b0, b1, b2, b3);
+    mma_bf16(s[0], a, b0, b1);
+    mma_bf16(s[1], a, b2, b3);
+  }
+}
+
 // O (16 x D) += P (16 x 16, A fragment) . T (16 x D tile at vt): rows of T
 // are the contraction index.
 template <int D>
