@@ -85,7 +85,7 @@ def algorithmic_work(w: workloads.Workload) -> dict:
 def launches_per_step(L: int) -> dict:
     """Kernels each entry point launches (matches the C library's dispatch)."""
     return {"pool": 1 + max(0, L - 2), "select": L, "fwd": 1, "transpose": 1,
-            "bwd": 2 + max(0, L - 1)}
+            "bwd": 2 + max(0, L - 1) + max(0, L - 2)}
 
 
 # ---------------------------------------------------------------- clocks

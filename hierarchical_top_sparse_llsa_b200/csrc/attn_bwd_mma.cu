@@ -57,7 +57,7 @@ __device__ __forceinline__ void probs_rows(const float (&s)[2][4], const float (
     for (int e = 0; e < 4; ++e) {
       const float lse = (e < 2) ? lse_g : lse_g8;
       const float x = fmaf(s[nt][e], sc2, lw[nt][e & 1] - lse);
-      P[nt][e] = (lse == -INFINITY) ? 0.f : exp2f(x);
+      P[nt][e] = (lse == -INFINITY) ? 0.f : ex2_approx(x);
     }
   }
 }
@@ -535,7 +535,7 @@ bwd_kv_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
       for (int e = 0; e < 4; ++e) {
         const int qi = 8 * nt + 2 * t + (e & 1);
         const float l2 = side[qi] * kLog2e;
-        P[nt][e] = (l2 == -INFINITY) ? 0.f : exp2f(fmaf(s_cur[nt][e], sc2, -l2));
+        P[nt][e] = (l2 == -INFINITY) ? 0.f : ex2_approx(fmaf(s_cur[nt][e], sc2, -l2));
         dS[nt][e] = P[nt][e] * (d_cur[nt][e] - side[16 + qi]);
       }
     uint32_t ph[4], pl[4], dsh[4], dsl[4];

@@ -202,6 +202,7 @@ __global__ void bwd_coarse_reduce_kernel(AttnParams p, int l) {
   const int nl = p.N >> (4 * l);
   const int NG = p.N >> 7;
   const int span = 2 << (4 * (l - 2));  // groups of 8 query blocks under a level-l token
+  const int nsum = (l >= 3) ? 1 : span;  // levels >= 3 were pre-added into the first group
   const int t = threadIdx.x;            // kv * D + d
   const int32_t* rp = p.row_ptr[l] + (size_t)bh * (nl + 1);
   const int32_t* col = p.col[l] + (size_t)bh * nl * K;
@@ -228,7 +229,7 @@ __global__ void bwd_coarse_reduce_kernel(AttnParams p, int l) {
       const float* src = part + ((size_t)s_q[e] * span * K + slot) * 2 * D;
       const size_t stride = (size_t)K * 2 * D;  // next group, same slot
       int a = 0;
-      for (; a + 4 <= span; a += 4) {
+      for (; a + 4 <= nsum; a += 4) {
         const float x0 = src[(a + 0) * stride], x1 = src[(a + 1) * stride];
         const float x2 = src[(a + 2) * stride], x3 = src[(a + 3) * stride];
         acc += x0;
@@ -236,7 +237,7 @@ __global__ void bwd_coarse_reduce_kernel(AttnParams p, int l) {
         acc += x2;
         acc += x3;
       }
-      for (; a < span; ++a) acc += src[a * stride];
+      for (; a < nsum; ++a) acc += src[a * stride];
     }
   }
   p.coarse[l][((size_t)bh * nl + c) * 2 * D + t] = acc;
@@ -353,8 +354,38 @@ cudaError_t launch_typed(const AttnParams& p, cudaStream_t s) {
 
 }  // namespace
 
+// For levels >= 3, first add each level-l query token's groups into its first
+// group (thread per (token, slot, kv, d); the groups in ascending order), so
+// the key-major gather reads one group per entry.
+__global__ void bwd_span_reduce_kernel(AttnParams p, int l) {
+  const int D = p.D, K = p.K;
+  const int nl = p.N >> (4 * l);
+  const int NG = p.N >> 7;
+  const int span = 2 << (4 * (l - 2));
+  const size_t per_tok = (size_t)K * 2 * D;
+  const size_t total = (size_t)p.B * p.H * nl * per_tok;
+  for (size_t e = (size_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+       e += (size_t)gridDim.x * blockDim.x) {
+    const size_t w = e % per_tok;
+    const size_t tok = e / per_tok;  // bh * nl + ql
+    const size_t bh = tok / nl, ql = tok % nl;
+    float* first = p.part[l] + ((bh * NG + ql * span) * per_tok) + w;
+    float acc = first[0];
+    for (int a = 1; a < span; ++a) acc += first[(size_t)a * per_tok];
+    first[0] = acc;
+  }
+}
+
 cudaError_t launch_coarse_reduce(const AttnParams& p, cudaStream_t s) {
   for (int l = 2; l <= p.L; ++l) {
+    if (l >= 3) {
+      const size_t total = (size_t)p.B * p.H * (p.N >> (4 * l)) * p.K * 2 * p.D;
+      int blocks = (int)((total + 255) / 256);
+      if (blocks > 148 * 16) blocks = 148 * 16;
+      bwd_span_reduce_kernel<<<blocks, 256, 0, s>>>(p, l);
+      const cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
     bwd_coarse_reduce_kernel<<<dim3(p.N >> (4 * l), p.B * p.H), 2 * p.D, 0, s>>>(p, l);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;

@@ -32,14 +32,20 @@ constexpr int kStages = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
+// Probabilities are taken relative to a reference max m_ref per row that is
+// only raised when the running max exceeds it by more than kRescaleLog2 (so
+// p <= 2^8): the output accumulators are rescaled rarely, and only when some
+// row of the warp needs it (FlashAttention-4's conditional rescaling).
+constexpr float kRescaleLog2 = 8.0f;
+
 struct SoftmaxState {
-  float m[2];  // running max of rows g and g+8 (base-2 scaled scores)
-  float l[2];  // this thread's partial row sums
+  float m[2];  // reference max of rows g and g+8 (base-2 scaled scores)
+  float l[2];  // this thread's partial row sums, relative to m
 };
 
 // Online-softmax update of a 16x16 score tile held in two m16n8 accumulators
 // (s[nt][0..1]: row g, keys 8nt+2t, 8nt+2t+1; s[nt][2..3]: row g+8), then
-// P (bf16 A fragment) and rescaling of the output accumulators.
+// P (bf16 A fragment) and rescaling of the output accumulators when needed.
 template <int NT>
 __device__ __forceinline__ void softmax_tile(float (&s)[2][4], const float (&lw)[2][2], float sc2,
                                              SoftmaxState& st, float (&o)[NT][4],
@@ -52,37 +58,50 @@ __device__ __forceinline__ void softmax_tile(float (&s)[2][4], const float (&lw)
     x[nt][2] = fmaf(s[nt][2], sc2, lw[nt][0]);
     x[nt][3] = fmaf(s[nt][3], sc2, lw[nt][1]);
   }
-  float mx0 = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
-  float mx1 = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
-  mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-  mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-  mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-  mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-  const float mn0 = fmaxf(st.m[0], mx0), mn1 = fmaxf(st.m[1], mx1);
-  // a row whose every score so far is -inf keeps corr = 1 and p = 0
-  const float c0 = (mn0 == -INFINITY) ? 1.f : exp2f(st.m[0] - mn0);
-  const float c1 = (mn1 == -INFINITY) ? 1.f : exp2f(st.m[1] - mn1);
-  const float b0 = (mn0 == -INFINITY) ? 0.f : mn0;
-  const float b1 = (mn1 == -INFINITY) ? 0.f : mn1;
+  // common path: no max at all, only a check that no score exceeds the
+  // reference by more than the threshold (false while the reference is -inf
+  // only if the tile is fully masked too)
+  bool hi = false;
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt)
+    hi |= (x[nt][0] > st.m[0] + kRescaleLog2) | (x[nt][1] > st.m[0] + kRescaleLog2) |
+          (x[nt][2] > st.m[1] + kRescaleLog2) | (x[nt][3] > st.m[1] + kRescaleLog2);
+  if (__any_sync(0xffffffffu, hi)) {
+    float mx0 = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
+    float mx1 = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    const bool up0 = mx0 > st.m[0] + kRescaleLog2;
+    const bool up1 = mx1 > st.m[1] + kRescaleLog2;
+    const float c0 = up0 ? ex2_approx(st.m[0] - mx0) : 1.f;  // 2^-inf = 0 for a first max
+    const float c1 = up1 ? ex2_approx(st.m[1] - mx1) : 1.f;
+    if (up0) st.m[0] = mx0;
+    if (up1) st.m[1] = mx1;
+    st.l[0] *= c0;
+    st.l[1] *= c1;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      o[nt][0] *= c0;
+      o[nt][1] *= c0;
+      o[nt][2] *= c1;
+      o[nt][3] *= c1;
+    }
+  }
+  // a row whose every score so far is -inf keeps m = -inf and gets p = 0
+  const float b0 = (st.m[0] == -INFINITY) ? 0.f : st.m[0];
+  const float b1 = (st.m[1] == -INFINITY) ? 0.f : st.m[1];
   float p[2][4];
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt) {
-    p[nt][0] = exp2f(x[nt][0] - b0);
-    p[nt][1] = exp2f(x[nt][1] - b0);
-    p[nt][2] = exp2f(x[nt][2] - b1);
-    p[nt][3] = exp2f(x[nt][3] - b1);
+    p[nt][0] = ex2_approx(x[nt][0] - b0);
+    p[nt][1] = ex2_approx(x[nt][1] - b0);
+    p[nt][2] = ex2_approx(x[nt][2] - b1);
+    p[nt][3] = ex2_approx(x[nt][3] - b1);
   }
-  st.l[0] = st.l[0] * c0 + (p[0][0] + p[0][1] + p[1][0] + p[1][1]);
-  st.l[1] = st.l[1] * c1 + (p[0][2] + p[0][3] + p[1][2] + p[1][3]);
-  st.m[0] = mn0;
-  st.m[1] = mn1;
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    o[nt][0] *= c0;
-    o[nt][1] *= c0;
-    o[nt][2] *= c1;
-    o[nt][3] *= c1;
-  }
+  st.l[0] += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
+  st.l[1] += (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]);
   pa[0] = pack_bf16(p[0][0], p[0][1]);
   pa[1] = pack_bf16(p[0][2], p[0][3]);
   pa[2] = pack_bf16(p[1][0], p[1][1]);

@@ -5,9 +5,10 @@
 // One launch per level, coarsest first.  A CTA owns the 16 sibling query
 // tokens under one parent (level l < L), or 16 consecutive query tokens at
 // the top level, so they share one candidate list: the children of the keys
-// their parent kept, or every top-level key.  Candidate K(l) rows are staged
-// in shared memory once per CTA in chunks of 128 and scored by 16 warps, one
-// query per warp, one candidate per lane.
+// their parent kept, or every top-level key.  Query rows and candidate K(l)
+// rows (in chunks of 128) are staged transposed in shared memory, and each
+// thread scores a 4 x 4 block of (query, candidate) pairs, so a candidate row
+// is read from shared memory 4 times rather than 16.
 //
 // Score: fp32, d = 0..D-1 left to right, one rounding per multiply and per
 // add (explicit __fmul_rn/__fadd_rn: no contraction into FMA), so scores are
@@ -23,8 +24,10 @@ namespace llsa {
 
 namespace {
 
-constexpr int kSelWarps = 16;
-constexpr int kSelChunk = 128;
+constexpr int kSelQ = 16;        // sibling query tokens per CTA
+constexpr int kSelWarps = 4;
+constexpr int kSelThreads = kSelWarps * 32;
+constexpr int kSelChunk = 128;   // candidates scored per pass
 constexpr int kSelItems = kSelChunk / 32;
 
 __device__ __forceinline__ uint64_t pack_key(float s, int idx) {
@@ -42,127 +45,155 @@ __device__ __forceinline__ uint64_t warp_max_u64(uint64_t x) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(kSelWarps * 32)
+__global__ void __launch_bounds__(kSelThreads)
 select_kernel(SelectParams p) {
-  constexpr int LD = D + 4;  // row stride (floats): conflict-free 16-byte loads
+  constexpr int QLD = kSelQ;            // queries per CTA, row stride of qsT
+  constexpr int CLD = kSelChunk + 4;    // row stride of ksT (floats)
   extern __shared__ float4 smem4[];
-  float* qs = reinterpret_cast<float*>(smem4);     // [16][LD]
-  float* ks = qs + kSelWarps * LD;                 // [kSelChunk][LD]
-  int* cid = reinterpret_cast<int*>(ks + kSelChunk * LD);  // [kSelChunk]
+  float* qsT = reinterpret_cast<float*>(smem4);   // [D][16] queries, transposed
+  float* ksT = qsT + D * QLD;                     // [D][CLD] candidates, transposed
+  float* sc = ksT + D * CLD;                      // [16][kSelChunk] scores of a chunk
+  int* cid = reinterpret_cast<int*>(sc + kSelQ * kSelChunk);  // [kSelChunk]
   __shared__ int parents[kMaxK];
   __shared__ int n_par;
 
   const int bh = blockIdx.y;
   const int grp = blockIdx.x;
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
   const int n = p.n;
   const int K = p.K;
   const bool top = (p.parent == nullptr);
 
-  if (threadIdx.x == 0) {
+  if (warp == 0) {
     int m = 0;
     if (!top) {
-      RowRule rr;
-      const int32_t* prow = p.parent + ((size_t)bh * (n / kBlock) + grp) * K;
-      for (int s = 0; s < K; ++s) {
-        const int c = prow[s];
-        if (rr.use(c, n / kBlock)) parents[m++] = c;
-      }
+      const int np = n / kBlock;
+      int f = 0;
+      const int c = (lane < K) ? p.parent[((size_t)bh * np + grp) * K + lane] : -1;
+      const bool u = warp_row_used(c, lane, np, lane < K, f);
+      const unsigned msk = __ballot_sync(0xffffffffu, u);
+      if (u) parents[__popc(msk & ((1u << lane) - 1u))] = c;
+      m = __popc(msk);
     }
-    n_par = m;
+    if (lane == 0) n_par = m;
   }
-  // the 16 query rows
-  const float* qbase = p.ql + ((size_t)bh * n + (size_t)grp * kSelWarps) * D;
-  for (int e = threadIdx.x; e < kSelWarps * (D / 4); e += blockDim.x) {
+  // the 16 query rows, transposed
+  const float* qbase = p.ql + ((size_t)bh * n + (size_t)grp * kSelQ) * D;
+  for (int e = tid; e < kSelQ * (D / 4); e += kSelThreads) {
     const int r = e / (D / 4), c4 = e % (D / 4);
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (grp * kSelWarps + r < n) v = *reinterpret_cast<const float4*>(qbase + (size_t)r * D + c4 * 4);
-    *reinterpret_cast<float4*>(qs + r * LD + c4 * 4) = v;
+    if (grp * kSelQ + r < n) v = *reinterpret_cast<const float4*>(qbase + (size_t)r * D + c4 * 4);
+    qsT[(4 * c4 + 0) * QLD + r] = v.x;
+    qsT[(4 * c4 + 1) * QLD + r] = v.y;
+    qsT[(4 * c4 + 2) * QLD + r] = v.z;
+    qsT[(4 * c4 + 3) * QLD + r] = v.w;
   }
   __syncthreads();
   const int C = top ? n : n_par * kBlock;
-  const int q = grp * kSelWarps + warp;
+  // this thread's 4 x 4 block of (query, candidate) scores
+  const int qg = tid >> 5;        // queries 4qg .. 4qg+3
+  const int cg = tid & 31;        // candidates 4cg .. 4cg+3 of a chunk
 
-  uint64_t run = 0;  // lane r < K holds the r-th best so far (0 = none)
+  uint64_t run[kSelQ / kSelWarps];  // per warp query: lane r < K holds its r-th best
+#pragma unroll
+  for (int i = 0; i < kSelQ / kSelWarps; ++i) run[i] = 0;
   const float* kbase = p.kl + (size_t)bh * n * D;
   for (int c0 = 0; c0 < C; c0 += kSelChunk) {
     const int cn = min(kSelChunk, C - c0);
     __syncthreads();
-    for (int e = threadIdx.x; e < cn * (D / 4); e += blockDim.x) {
-      const int r = e / (D / 4), c4 = e % (D / 4);
-      const int j = c0 + r;
-      const int c = top ? j : parents[j / kBlock] * kBlock + (j % kBlock);
-      *reinterpret_cast<float4*>(ks + r * LD + c4 * 4) =
-          *reinterpret_cast<const float4*>(kbase + (size_t)c * D + c4 * 4);
-      if (c4 == 0) cid[r] = c;
+    for (int e = tid; e < kSelChunk * (D / 4); e += kSelThreads) {
+      const int r = e % kSelChunk, c4 = e / kSelChunk;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (r < cn) {
+        const int j = c0 + r;
+        const int c = top ? j : parents[j / kBlock] * kBlock + (j % kBlock);
+        v = *reinterpret_cast<const float4*>(kbase + (size_t)c * D + c4 * 4);
+        if (c4 == 0) cid[r] = c;
+      }
+      ksT[(4 * c4 + 0) * CLD + r] = v.x;
+      ksT[(4 * c4 + 1) * CLD + r] = v.y;
+      ksT[(4 * c4 + 2) * CLD + r] = v.z;
+      ksT[(4 * c4 + 3) * CLD + r] = v.w;
     }
     __syncthreads();
-    uint64_t item[kSelItems + 1];
+    // scores: d = 0..D-1 in order, one rounding per multiply and per add
+    float acc[4][4];
 #pragma unroll
-    for (int it = 0; it < kSelItems; ++it) {
-      const int j = lane + 32 * it;
-      item[it] = 0;
-      if (j < cn) {
-        const float* qr = qs + warp * LD;
-        const float* kr = ks + j * LD;
-        float s = 0.f;
+    for (int d = 0; d < D; ++d) {
+      const float4 qv = *reinterpret_cast<const float4*>(qsT + d * QLD + 4 * qg);
+      const float4 kv = *reinterpret_cast<const float4*>(ksT + d * CLD + 4 * cg);
+      const float qq[4] = {qv.x, qv.y, qv.z, qv.w};
+      const float kk[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
-        for (int d = 0; d < D; d += 4) {
-          const float4 a = *reinterpret_cast<const float4*>(qr + d);
-          const float4 b = *reinterpret_cast<const float4*>(kr + d);
-          s = (d == 0) ? __fmul_rn(a.x, b.x) : __fadd_rn(s, __fmul_rn(a.x, b.x));
-          s = __fadd_rn(s, __fmul_rn(a.y, b.y));
-          s = __fadd_rn(s, __fmul_rn(a.z, b.z));
-          s = __fadd_rn(s, __fmul_rn(a.w, b.w));
-        }
-        item[it] = pack_key(s, cid[j]);
-      }
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          acc[a][c] = (d == 0) ? __fmul_rn(qq[a], kk[c]) : __fadd_rn(acc[a][c], __fmul_rn(qq[a], kk[c]));
     }
-    item[kSelItems] = (lane < K) ? run : 0;
-    uint64_t next = 0;
-    for (int r = 0; r < K; ++r) {
-      uint64_t mine = 0;
-      int arg = 0;
 #pragma unroll
-      for (int it = 0; it <= kSelItems; ++it)
-        if (item[it] > mine) { mine = item[it]; arg = it; }
-      const uint64_t best = warp_max_u64(mine);
-      if (best == 0) break;  // uniform: no candidates left
-      if (mine == best) {
+    for (int a = 0; a < 4; ++a)
+      *reinterpret_cast<float4*>(sc + (4 * qg + a) * kSelChunk + 4 * cg) =
+          make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+    __syncthreads();
+    // Top-K merge, one query of this warp at a time
+#pragma unroll
+    for (int qi = 0; qi < kSelQ / kSelWarps; ++qi) {
+      const int ql = warp * (kSelQ / kSelWarps) + qi;
+      uint64_t item[kSelItems + 1];
+#pragma unroll
+      for (int it = 0; it < kSelItems; ++it) {
+        const int j = lane + 32 * it;
+        item[it] = (j < cn) ? pack_key(sc[ql * kSelChunk + j], cid[j]) : 0;
+      }
+      item[kSelItems] = (lane < K) ? run[qi] : 0;
+      uint64_t next = 0;
+      for (int r = 0; r < K; ++r) {
+        uint64_t mine = 0;
+        int arg = 0;
 #pragma unroll
         for (int it = 0; it <= kSelItems; ++it)
-          if (it == arg) item[it] = 0;
+          if (item[it] > mine) { mine = item[it]; arg = it; }
+        const uint64_t best = warp_max_u64(mine);
+        if (best == 0) break;  // uniform: no candidates left
+        if (mine == best) {
+#pragma unroll
+          for (int it = 0; it <= kSelItems; ++it)
+            if (it == arg) item[it] = 0;
+        }
+        if (lane == r) next = best;
       }
-      if (lane == r) next = best;
+      run[qi] = next;
     }
-    run = next;
   }
-  if (q >= n) return;
   // ascending index order; the kept entries are lanes 0..cnt-1
-  const bool valid = (lane < K) && (run != 0);
-  const int id = valid ? (int)(~(uint32_t)run) : 0x7fffffff;
-  int pos = 0;
-  for (int r = 0; r < K; ++r) {
-    const int other = __shfl_sync(0xffffffffu, id, r);
-    pos += (other < id) ? 1 : 0;
-  }
-  if (lane < K) {
-    int32_t* orow = p.out + ((size_t)bh * n + q) * K;
-    if (valid) orow[pos] = id;
-    else orow[lane] = -1;  // unfilled rounds are the last K - cnt lanes
+#pragma unroll
+  for (int qi = 0; qi < kSelQ / kSelWarps; ++qi) {
+    const int q = grp * kSelQ + warp * (kSelQ / kSelWarps) + qi;
+    const bool valid = (lane < K) && (run[qi] != 0);
+    const int id = valid ? (int)(~(uint32_t)run[qi]) : 0x7fffffff;
+    int pos = 0;
+    for (int r = 0; r < K; ++r) {
+      const int other = __shfl_sync(0xffffffffu, id, r);
+      pos += (other < id) ? 1 : 0;
+    }
+    if (q < n && lane < K) {
+      int32_t* orow = p.out + ((size_t)bh * n + q) * K;
+      if (valid) orow[pos] = id;
+      else orow[lane] = -1;  // unfilled rounds are the last K - cnt lanes
+    }
   }
 }
 
 template <int D>
 cudaError_t launch_sel(const SelectParams& p, int BH, cudaStream_t s) {
-  constexpr int LD = D + 4;
-  const size_t smem = (size_t)(kSelWarps + kSelChunk) * LD * sizeof(float) + kSelChunk * sizeof(int);
+  const size_t smem = (size_t)(D * kSelQ + D * (kSelChunk + 4) + kSelQ * kSelChunk) * sizeof(float) +
+                      kSelChunk * sizeof(int);
   // set on every call: the attribute is per device and the call is cheap
   cudaError_t e = cudaFuncSetAttribute(select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const int groups = (p.parent == nullptr) ? (p.n + kSelWarps - 1) / kSelWarps : p.n / kBlock;
-  select_kernel<D><<<dim3(groups, BH), kSelWarps * 32, smem, s>>>(p);
+  const int groups = (p.parent == nullptr) ? (p.n + kSelQ - 1) / kSelQ : p.n / kBlock;
+  select_kernel<D><<<dim3(groups, BH), kSelThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
 

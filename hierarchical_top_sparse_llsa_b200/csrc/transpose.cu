@@ -25,6 +25,7 @@ namespace {
 
 constexpr int kTrWarps = 16;
 constexpr int kTrRange = 256;
+constexpr int kBatch = 8;  // row steps whose index loads are in flight together
 
 __global__ void __launch_bounds__(kTrWarps * 32)
 transpose_kernel(TransposeParams p) {
@@ -59,15 +60,25 @@ transpose_kernel(TransposeParams p) {
   const int rpw = (n + kTrWarps - 1) / kTrWarps;  // rows per warp
   const int r_begin = min(n, warp * rpw), r_end = min(n, r_begin + rpw);
 
-  // pass 1: counts
+  // pass 1: counts (entries of kBatch steps are loaded before any is used,
+  // so their latencies overlap)
   int flags = 0, my_below = 0;
-  for (int r0 = r_begin; r0 < r_end; r0 += rows_per_step) {
-    const int q = r0 + sub;
-    const bool on = lane_on && q < r_end;
-    const int c = on ? I[(size_t)q * K + slot] : -1;
-    const bool u = warp_row_used(c, slot, n, on, flags);
-    if (u && c >= c0 && c < c1) atomicAdd(&hist[warp][c - c0], 1);
-    if (u && c < c0) ++my_below;
+  for (int rb = r_begin; rb < r_end; rb += kBatch * rows_per_step) {
+    int cb[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int q = rb + i * rows_per_step + sub;
+      cb[i] = (lane_on && q < r_end) ? I[(size_t)q * K + slot] : -1;
+    }
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int q = rb + i * rows_per_step + sub;
+      const bool on = lane_on && q < r_end;
+      const int c = cb[i];
+      const bool u = warp_row_used(c, slot, n, on, flags);
+      if (u && c >= c0 && c < c1) atomicAdd(&hist[warp][c - c0], 1);
+      if (u && c < c0) ++my_below;
+    }
   }
   my_below = __reduce_add_sync(0xffffffffu, my_below);
   if (lane == 0) below[warp] = my_below;
@@ -117,22 +128,29 @@ transpose_kernel(TransposeParams p) {
 
   // pass 2: fill
   int dummy = 0;
-  for (int r0 = r_begin; r0 < r_end; r0 += rows_per_step) {
-    const int q = r0 + sub;
-    const bool on = lane_on && q < r_end;
-    const int c = on ? I[(size_t)q * K + slot] : -1;
-    const bool u = warp_row_used(c, slot, n, on, dummy);
-    const int key = (u && c >= c0 && c < c1) ? c : -2 - lane;  // -2 - lane matches nobody
-    const unsigned peers = __match_any_sync(0xffffffffu, key);
-    int pos = 0;
-    if (key >= 0) {
-      const unsigned lower = peers & ((1u << lane) - 1u);
-      pos = hist[warp][key - c0] + __popc(lower);
-      col[pos] = q;
+  for (int rb = r_begin; rb < r_end; rb += kBatch * rows_per_step) {
+    int cb[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int q = rb + i * rows_per_step + sub;
+      cb[i] = (lane_on && q < r_end) ? I[(size_t)q * K + slot] : -1;
     }
-    __syncwarp();
-    if (key >= 0 && lane == 31 - __clz(peers)) hist[warp][key - c0] += __popc(peers);
-    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int q = rb + i * rows_per_step + sub;
+      const bool on = lane_on && q < r_end;
+      const int c = cb[i];
+      const bool u = warp_row_used(c, slot, n, on, dummy);
+      const int key = (u && c >= c0 && c < c1) ? c : -2 - lane;  // -2 - lane matches nobody
+      const unsigned peers = __match_any_sync(0xffffffffu, key);
+      if (key >= 0) {
+        const unsigned lower = peers & ((1u << lane) - 1u);
+        col[hist[warp][key - c0] + __popc(lower)] = q;
+      }
+      __syncwarp();
+      if (key >= 0 && lane == 31 - __clz(peers)) hist[warp][key - c0] += __popc(peers);
+      __syncwarp();
+    }
   }
   if (local % L.ranges == 0) {
     flags = __reduce_or_sync(0xffffffffu, flags);
