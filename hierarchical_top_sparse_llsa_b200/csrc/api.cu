@@ -13,12 +13,17 @@ namespace llsa {
 cudaError_t launch_attn_fwd_simt(const AttnParams& p, int dtype, cudaStream_t s);
 cudaError_t launch_attn_bwd_simt(const AttnParams& p, int dtype, cudaStream_t s);
 cudaError_t launch_attn_fwd_mma(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s);
+cudaError_t launch_attn_fwd_tc(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s);
 cudaError_t launch_attn_bwd_mma(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s);
 }  // namespace llsa
 
 using namespace llsa;
 
 namespace {
+
+// The tcgen05 forward (attn_fwd_tc.cu) is parity-green but not yet faster
+// than the warp-MMA forward, which therefore stays the bf16 default.
+constexpr bool kUseTcForward = false;
 
 inline int check_desc(const llsa_desc* d) {
   if (d == nullptr) return LLSA_ERR_INVALID_ARG;
@@ -230,6 +235,8 @@ int llsa_attn_fwd(const llsa_desc* desc, const void* q, const void* k, const voi
     st = make_row_tile_map(&maps[i], srcs[i], rows, desc->D);
     if (st != LLSA_OK) return st;
   }
+  if (kUseTcForward && desc->D == 64)  // tcgen05 MMAs into tensor memory
+    return launch_status(launch_attn_fwd_tc(p, maps, (cudaStream_t)stream));
   return launch_status(launch_attn_fwd_mma(p, maps, (cudaStream_t)stream));
 }
 
