@@ -239,7 +239,8 @@ def run_ours(args, rank, world, local_rank):
     t_in = {k: torch.from_numpy(v).to(dev, dtype=tdt) for k, v in x.items()}
     host = {k: torch.from_numpy(v).to(dtype=tdt).pin_memory() for k, v in x.items()}
     del x
-    desc = llsa.make_desc(w.B, w.H, w.N, w.D, w.L, w.topk, llsa.BF16 if w.dtype == "bf16" else llsa.F32)
+    desc = llsa.make_desc(w.B, w.H, w.N, w.D, w.L, w.topk, llsa.BF16 if w.dtype == "bf16" else llsa.F32,
+                          flags=llsa.FLAG_FWD_TCGEN05 if args.fwd_tcgen05 else 0)
     bufs = llsa.LlsaBuffers(desc, dev, with_bwd=w.backward)
     o = torch.empty_like(t_in["q"])
     lse = torch.empty(w.B, w.H, w.N, dtype=torch.float32, device=dev)
@@ -399,6 +400,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=workloads.HEADLINE, choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fwd-tcgen05", action="store_true",
+                    help="run the forward on the tcgen05 kernel (bf16, D=64)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be at least 3")

@@ -27,6 +27,7 @@ BLOCK = 16
 F32, BF16 = 0, 1
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_LAUNCH, ERR_WORKSPACE = 0, 1, 2, 3, 4
 DEV_BAD_INDEX, DEV_NONCANONICAL, DEV_TIMEOUT = 1, 2, 4
+FLAG_FWD_TCGEN05 = 1
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 EXPORTED = (
@@ -110,12 +111,12 @@ def _check(status: int) -> int:
     return status
 
 
-def make_desc(B, H, N, D, L, topk, dtype, sm_scale=0.0, level_w=None) -> LlsaDesc:
+def make_desc(B, H, N, D, L, topk, dtype, sm_scale=0.0, level_w=None, flags=0) -> LlsaDesc:
     """Fill an llsa_desc; level_w is None (every weight 1) or indexable by level."""
     d = LlsaDesc()
     d.B, d.H, d.N, d.D, d.L, d.topk = B, H, N, D, L, topk
     d.dtype = dtype
-    d.flags = 0
+    d.flags = flags
     d.sm_scale = sm_scale
     for l in range(MAX_LEVELS + 1):
         d.level_w[l] = 0.0

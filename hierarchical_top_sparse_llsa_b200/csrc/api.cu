@@ -21,15 +21,15 @@ using namespace llsa;
 
 namespace {
 
-// The tcgen05 forward (attn_fwd_tc.cu) is parity-green but not yet faster
-// than the warp-MMA forward, which therefore stays the bf16 default.
+// The tcgen05 forward (attn_fwd_tc.cu) is the bf16 D = 64 default only when
+// it is the faster of the two; LLSA_FLAG_FWD_TCGEN05 selects it explicitly.
 constexpr bool kUseTcForward = false;
 
 inline int check_desc(const llsa_desc* d) {
   if (d == nullptr) return LLSA_ERR_INVALID_ARG;
   if (d->B < 1 || d->H < 1 || d->N < kBlock || d->D < 1 || d->L < 1 || d->topk < 1)
     return LLSA_ERR_INVALID_ARG;
-  if (d->flags != 0) return LLSA_ERR_INVALID_ARG;
+  if ((d->flags & ~LLSA_FLAG_FWD_TCGEN05) != 0) return LLSA_ERR_INVALID_ARG;
   if (d->dtype != LLSA_F32 && d->dtype != LLSA_BF16) return LLSA_ERR_INVALID_ARG;
   if (d->D != 64 && d->D != 128) return LLSA_ERR_UNSUPPORTED;
   if (d->L > kMaxL || d->topk > kMaxK) return LLSA_ERR_UNSUPPORTED;
@@ -235,7 +235,8 @@ int llsa_attn_fwd(const llsa_desc* desc, const void* q, const void* k, const voi
     st = make_row_tile_map(&maps[i], srcs[i], rows, desc->D);
     if (st != LLSA_OK) return st;
   }
-  if (kUseTcForward && desc->D == 64)  // tcgen05 MMAs into tensor memory
+  const bool use_tc = kUseTcForward || (desc->flags & LLSA_FLAG_FWD_TCGEN05) != 0;
+  if (use_tc && desc->D == 64)  // tcgen05 MMAs into tensor memory
     return launch_status(launch_attn_fwd_tc(p, maps, (cudaStream_t)stream));
   return launch_status(launch_attn_fwd_mma(p, maps, (cudaStream_t)stream));
 }

@@ -33,10 +33,12 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
 // Probabilities are taken relative to a reference max m_ref per row that is
-// only raised when the running max exceeds it by more than kRescaleLog2 (so
-// p <= 2^8): the output accumulators are rescaled rarely, and only when some
-// row of the warp needs it (FlashAttention-4's conditional rescaling).
-constexpr float kRescaleLog2 = 8.0f;
+// raised when a score exceeds it by more than kRescaleLog2; the output
+// accumulators are rescaled only when some row of the warp needs it.
+// Threshold 0: the reference is the exact running max, so the largest
+// probability of a row is exactly 1 and its bf16 rounding is exact; a lagging
+// reference (up to 2^8) let that rounding error through on rows with few keys.
+constexpr float kRescaleLog2 = 0.0f;
 
 struct SoftmaxState {
   float m[2];  // reference max of rows g and g+8 (base-2 scaled scores)

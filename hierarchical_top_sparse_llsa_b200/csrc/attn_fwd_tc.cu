@@ -9,14 +9,13 @@
 // blocks (64 keys): each chunk's K and V tiles arrive by 2D TMA loads
 // (128-byte swizzle, no multicast) into a double buffer, then
 //   S = Q K_chunk^T        (M 128, N <= 64, K 64) into tensor memory,
-//   P = 2^(S*scale - m)    by the 128 threads, one query row each, with the
+//   P = 2^(S*scale - m)    by 256 threads, two per query row, with the
 //                          key blocks its own query block did not select
 //                          masked out; P is written as bf16 to shared memory,
 //   O += P V_chunk         (M 128, N 64, K <= 64) accumulated in tensor memory.
 // The MMAs are issued by one thread and complete on mbarriers; the softmax
-// works on whole rows in registers (no shuffles), against a reference maximum
-// that is raised only when a score exceeds it by 2^8, in which case the row of
-// O is rescaled in tensor memory.  The coarse keys, shared by all 8 blocks,
+// works on half rows in registers (no shuffles), against the running row
+// maximum; when it grows, the row of O is rescaled in tensor memory.  The coarse keys, shared by all 8 blocks,
 // follow as padded chunks converted from the fp32 pyramid.  Key blocks a row
 // did not select cost MMA work but no exponentials; the union keeps that
 // waste near |U| / K per block instead of every candidate.
@@ -32,7 +31,8 @@ namespace llsa {
 namespace {
 
 constexpr int kTcBlocks = 8;      // query blocks per CTA (128 rows)
-constexpr int kTcThreads = 128;   // one thread per query row
+constexpr int kTcWarps = 8;
+constexpr int kTcThreads = kTcWarps * 32;  // two threads per query row (32 columns each)
 constexpr int kChunkBlocks = 4;   // key blocks per chunk (64 keys)
 constexpr int kTcD = 64;
 constexpr int kTile = 32 * kTcD;  // bytes of a 16-row bf16 tile (2 KB)
@@ -40,7 +40,10 @@ constexpr int kMaxUnion = kTcBlocks * kMaxK;  // 256
 constexpr uint32_t kTmemCols = 128;           // S: columns 0..63, O: 64..127
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kRescaleLog2 = 8.0f;
+// Threshold 0: the reference is the exact running max, so the largest
+// probability of a row is exactly 1 and its bf16 rounding is exact; a lagging
+// reference (up to 2^8) let that rounding error through on rows with few keys.
+constexpr float kRescaleLog2 = 0.0f;
 
 // shared-memory layout (bytes from a 1024-aligned base)
 constexpr int kOffQ = 0;                                        // 8 tiles
@@ -58,6 +61,7 @@ struct TcShared {
   uint32_t mask[kTcBlocks][kMaxUnion / 32];  // block b selected union entry u
   int clist[kMaxL * kMaxK];           // coarse keys: level << 24 | token
   float clw[kMaxL * kMaxK + 64];      // their log2 weights (-inf for pads)
+  float red[2][128];                  // per row and column half: max, then sum
 };
 
 template <int E>
@@ -76,9 +80,9 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
   const size_t rowbase = (size_t)bh * p.N;
   int flags = 0;
 
-  // ---- selections of the 8 blocks (2 per warp), coarse list (warp 0)
-  for (int i = 0; i < kTcBlocks / 4; ++i) {
-    const int bi = warp * (kTcBlocks / 4) + i;
+  // ---- selections of the 8 blocks (one per warp), coarse list (warp 0)
+  for (int i = 0; i < kTcBlocks / kTcWarps; ++i) {
+    const int bi = warp * (kTcBlocks / kTcWarps) + i;
     const int b = b0 + bi;
     const bool on = (b < n1) && lane < K;
     const int v = on ? p.idx[1][((size_t)bh * n1 + b) * K + lane] : -1;
@@ -162,12 +166,15 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
     S.clw[e] = (e < nc) ? p.logw[S.clist[e] >> 24] * kLog2e : -INFINITY;
   __syncthreads();  // membership masks and coarse weights complete
 
-  // this thread's query row
-  const int r = tid;                 // TMEM lane r, P row r
-  const int qb = r >> 4;             // its query block within the CTA
-  const uint32_t t_row = (uint32_t)(warp * 32) << 16;  // lane field of this warp's quarter
+  // this thread's query row and column half: warp w may only touch TMEM
+  // lanes 32 (w % 4) .. +31
+  const int quarter = warp & 3, half = warp >> 2;
+  const int r = quarter * 32 + lane;       // TMEM lane r, P row r
+  const int qb = r >> 4;                   // its query block within the CTA
+  const uint32_t t_row = (uint32_t)(quarter * 32) << 16;
+  const int col0 = 32 * half;              // this thread's 32 of the 64 chunk columns
   const float sc2 = p.scale * kLog2e;
-  float m_ref = -INFINITY, lsum = 0.f;
+  float m_ref = -INFINITY, lsum = 0.f;     // lsum: this half's part of the row sum
   bool ok = mbar_wait_bounded(bq, 0);
   const uint32_t idesc_pv = idesc_bf16_f32(128, 64, 1);
 
@@ -213,68 +220,68 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
     }
     if (ok) ok = mbar_wait_bounded(bs, (uint32_t)(c & 1));
     tc_fence_after();
-    float s[64];
-    tmem_ld32(t_s + t_row, *reinterpret_cast<float(*)[32]>(&s[0]));
-    tmem_ld32(t_s + t_row + 32, *reinterpret_cast<float(*)[32]>(&s[32]));
+    float x[32];
+    tmem_ld32(t_s + t_row + col0, x);
     tmem_wait_ld();
     // (C) the previous PV has finished: O is stable, P and the other buffer are free
     if (c > 0 && ok) ok = mbar_wait_bounded(bpv, (uint32_t)((c - 1) & 1));
     tc_fence_after();
     // (D) prefetch the next fine chunk into the buffer just freed
     if (tid == 0 && ok && c + 1 < nfc && c + 1 >= 2) issue_fine(c + 1);
-    // (E) scores -> probabilities of this row
-    float x[64];
+    // (E) scores -> probabilities of this half row
     if (c < nfc) {
       const int u0 = c * kChunkBlocks;
       const uint32_t bits = (S.mask[qb][u0 >> 5] >> (u0 & 31)) & 0xFu;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const bool sel = (i < nb) && ((bits >> i) & 1u);
+      for (int i = 0; i < 2; ++i) {
+        const int blk = 2 * half + i;  // key block of the chunk for columns 16i..16i+15
+        const bool sel = (blk < nb) && ((bits >> blk) & 1u);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) x[16 * i + j] = sel ? s[16 * i + j] * sc2 : -INFINITY;
+        for (int j = 0; j < 16; ++j) x[16 * i + j] = sel ? x[16 * i + j] * sc2 : -INFINITY;
       }
     } else {
-      const int k0 = (c - nfc) * 64;
+      const int k0 = (c - nfc) * 64 + col0;
 #pragma unroll
-      for (int j = 0; j < 64; ++j) x[j] = fmaf(s[j], sc2, S.clw[k0 + j]);
+      for (int j = 0; j < 32; ++j) x[j] = fmaf(x[j], sc2, S.clw[k0 + j]);
     }
     bool hi = false;
 #pragma unroll
-    for (int j = 0; j < 64; ++j) hi |= x[j] > m_ref + kRescaleLog2;
-    if (__any_sync(0xffffffffu, hi)) {
+    for (int j = 0; j < 32; ++j) hi |= x[j] > m_ref + kRescaleLog2;
+    if (__syncthreads_or(hi)) {  // raise the running max of some rows
       float mx = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < 64; ++j) mx = fmaxf(mx, x[j]);
+      for (int j = 0; j < 32; ++j) mx = fmaxf(mx, x[j]);
+      S.red[half][r] = mx;
+      __syncthreads();
+      mx = fmaxf(S.red[0][r], S.red[1][r]);
       const bool up = mx > m_ref + kRescaleLog2;
       const float corr = up ? ex2_approx(m_ref - mx) : 1.f;  // 2^-inf = 0 for a first max
       if (up) m_ref = mx;
       lsum *= corr;
-      if (c > 0) {  // rescale this row of O (tensor memory, whole warp)
+      if (c > 0) {  // rescale this half row of O in tensor memory (whole warp)
         float o[32];
+        tmem_ld32(t_o + t_row + col0, o);
+        tmem_wait_ld();
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          tmem_ld32(t_o + t_row + 32 * h, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) o[j] *= corr;
-          tmem_st32(t_o + t_row + 32 * h, o);
-        }
+        for (int j = 0; j < 32; ++j) o[j] *= corr;
+        tmem_st32(t_o + t_row + col0, o);
         tmem_wait_st();
       }
+      __syncthreads();  // S.red reused below
     }
     const float mb = (m_ref == -INFINITY) ? 0.f : m_ref;
     unsigned char* prow = sm + kOffP + r * 128;
 #pragma unroll
-    for (int j8 = 0; j8 < 8; ++j8) {
+    for (int jj = 0; jj < 4; ++jj) {
       float pv[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        pv[e] = ex2_approx(x[8 * j8 + e] - mb);
+        pv[e] = ex2_approx(x[8 * jj + e] - mb);
         lsum += pv[e];
       }
       const uint4 pk = make_uint4(pack_bf16(pv[0], pv[1]), pack_bf16(pv[2], pv[3]),
                                   pack_bf16(pv[4], pv[5]), pack_bf16(pv[6], pv[7]));
-      *reinterpret_cast<uint4*>(prow + ((j8 ^ (r & 7)) << 4)) = pk;
+      *reinterpret_cast<uint4*>(prow + (((4 * half + jj) ^ (r & 7)) << 4)) = pk;
     }
     fence_proxy_async_smem();
     tc_fence_before();
@@ -292,27 +299,27 @@ attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant
   tc_fence_after();
 
   // ---- epilogue: O = acc / l, LSE = ln(sum) = (m + log2 l) ln 2
-  float o[64];
-  tmem_ld32(t_o + t_row, *reinterpret_cast<float(*)[32]>(&o[0]));
-  tmem_ld32(t_o + t_row + 32, *reinterpret_cast<float(*)[32]>(&o[32]));
+  S.red[half][r] = lsum;
+  __syncthreads();
+  const float ltot = S.red[0][r] + S.red[1][r];
+  float o[32];
+  tmem_ld32(t_o + t_row + col0, o);
   tmem_wait_ld();
   const int b = b0 + qb;
   if (b < n1) {
-    const bool has = lsum > 0.f && nch > 0;
-    const float inv = has ? 1.f / lsum : 0.f;
+    const bool has = ltot > 0.f && nch > 0;
+    const float inv = has ? 1.f / ltot : 0.f;
     const size_t tok = rowbase + (size_t)b0 * 16 + r;
-    bf16* O = static_cast<bf16*>(p.out) + tok * kTcD;
+    bf16* O = static_cast<bf16*>(p.out) + tok * kTcD + col0;
 #pragma unroll
-    for (int j8 = 0; j8 < 8; ++j8) {
-      uint4 pk;
+    for (int jj = 0; jj < 4; ++jj) {
+      uint4 pk = make_uint4(0, 0, 0, 0);
       if (has)
-        pk = make_uint4(pack_bf16(o[8 * j8] * inv, o[8 * j8 + 1] * inv), pack_bf16(o[8 * j8 + 2] * inv, o[8 * j8 + 3] * inv),
-                        pack_bf16(o[8 * j8 + 4] * inv, o[8 * j8 + 5] * inv), pack_bf16(o[8 * j8 + 6] * inv, o[8 * j8 + 7] * inv));
-      else
-        pk = make_uint4(0, 0, 0, 0);
-      reinterpret_cast<uint4*>(O)[j8] = pk;
+        pk = make_uint4(pack_bf16(o[8 * jj] * inv, o[8 * jj + 1] * inv), pack_bf16(o[8 * jj + 2] * inv, o[8 * jj + 3] * inv),
+                        pack_bf16(o[8 * jj + 4] * inv, o[8 * jj + 5] * inv), pack_bf16(o[8 * jj + 6] * inv, o[8 * jj + 7] * inv));
+      reinterpret_cast<uint4*>(O)[jj] = pk;
     }
-    p.lse[tok] = has ? (m_ref + log2f(lsum)) * kLn2 : -INFINITY;
+    if (half == 0) p.lse[tok] = has ? (m_ref + log2f(ltot)) * kLn2 : -INFINITY;
   }
   if (!ok) flags |= LLSA_DEV_TIMEOUT;
   flags = __reduce_or_sync(0xffffffffu, flags);

@@ -61,6 +61,14 @@ enum {
   LLSA_ERR_WORKSPACE = 4    /* workspace smaller than llsa_bwd_workspace_bytes() */
 };
 
+/* descriptor flags */
+enum {
+  /* bf16, D = 64: run llsa_attn_fwd on the tcgen05 kernel (tensor-memory
+   * accumulators, 8 sibling query blocks per 128-row MMA) instead of the
+   * warp-MMA kernel.  Both compute the same result within bf16 rounding. */
+  LLSA_FLAG_FWD_TCGEN05 = 1
+};
+
 /* device status bits (OR-ed into *dev_status) */
 enum {
   LLSA_DEV_BAD_INDEX = 1,    /* an index entry outside [-1, N_l) was skipped */
@@ -74,7 +82,7 @@ typedef struct {
   int L;          /* number of pooled levels, 1 <= L <= LLSA_MAX_LEVELS */
   int topk;       /* K, kept keys per level, 1 <= K <= LLSA_MAX_TOPK */
   int dtype;      /* LLSA_F32 or LLSA_BF16 */
-  int flags;      /* reserved, must be 0 */
+  int flags;      /* LLSA_FLAG_* bits; other bits must be 0 */
   float sm_scale; /* softmax scale; 0 selects 1/sqrt(D) */
   /* level_w[l], l = 2..L: weight of the coarse keys of level l (KV
    * Reweighting; the paper's setting is 16^l).  0 selects 1.  Entries 0, 1 and

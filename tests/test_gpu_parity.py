@@ -160,3 +160,41 @@ def test_runs_are_bitwise_deterministic():
     b = run_gpu(w.B, w.H, w.N, w.D, w.L, w.topk, w.dtype, x)
     for key in ("O", "LSE", "dQ", "dK", "dV"):
         assert np.array_equal(a[key], b[key], equal_nan=True), key
+
+
+@pytest.mark.parametrize("name,heads", [
+    ("img64_bf16", None),
+    ("img128_bf16", [3]),
+    ("img256_bf16", [7]),
+])
+def test_tcgen05_forward(name, heads):
+    # the tcgen05 forward kernel, selected by LLSA_FLAG_FWD_TCGEN05
+    w = workloads.WORKLOADS[name]
+    x = workloads.make_inputs(w)
+    g = run_gpu(w.B, w.H, w.N, w.D, w.L, w.topk, w.dtype, x, bwd=False, flags=llsa.FLAG_FWD_TCGEN05)
+    assert g["status"] == 0
+    hs = slice(None) if heads is None else heads
+    xs = x if heads is None else {k: np.ascontiguousarray(v[:, heads]) for k, v in x.items()}
+    r = run_oracle(xs, w.L, w.topk, bwd=False)
+    _compare(w, g, r, hs, False)
+
+
+@pytest.mark.parametrize("flags", [0, llsa.FLAG_FWD_TCGEN05])
+def test_forward_external_indices_and_weights(flags):
+    B, H, N, D, L, K = 1, 2, 4096, 64, 3, 6
+    x = _small(27, B, H, N, D)
+    rng = np.random.default_rng(28)
+    ext = {}
+    for l in range(1, L + 1):
+        n = N // 16**l
+        I = rng.integers(-3, n + 3, size=(B, H, n, K)).astype(np.int32)
+        I[..., 0, :] = -1
+        ext[l] = I
+    clean = {}
+    for l in range(1, L + 1):
+        clean[l], _ = clean_indices(ext[l], N // 16**l)
+    lw = [0, 0, 16.0**2, 16.0**3]
+    g = run_gpu(B, H, N, D, L, K, "bf16", x, ext_idx=ext, bwd=False, level_w=lw, flags=flags)
+    r = run_oracle(x, L, K, idx=clean, bwd=False, level_w=lw)
+    assert_close(g["O"], r["O"], "bf16", "O")
+    assert_close(g["LSE"], r["LSE"], "bf16", "LSE")
