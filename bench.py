@@ -15,10 +15,12 @@ prints one JSON line.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import datetime
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -82,9 +84,90 @@ def algorithmic_work(w: workloads.Workload) -> dict:
     return work
 
 
+def sources_digest() -> str:
+    """sha1 over the library's CUDA sources: ties a committed ncu traffic
+    figure to the kernels it was measured on."""
+    h = hashlib.sha1()
+    csrc = os.path.join(ROOT, "hierarchical_top_sparse_llsa_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            h.update(name.encode())
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(f.read())
+    with open(os.path.join(ROOT, "include", "llsa.h"), "rb") as f:
+        h.update(f.read())
+    return h.hexdigest()
+
+
+def committed_traffic(workload: str, stage: str):
+    """DRAM bytes per call of `stage` from the committed ncu summary of this
+    workload, or None when there is none or the sources changed since."""
+    path = os.path.join(ROOT, "profiles", f"dram_traffic_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        text = f.read()
+    m = re.search(r"```json\n(.*?)\n```", text, re.S)
+    if m is None:
+        return None
+    rec = json.loads(m.group(1))
+    if rec.get("sources_sha1") != sources_digest():
+        return None
+    st = rec.get("stages", {}).get(stage)
+    return None if st is None else st.get("dram_bytes_per_call")
+
+
+def dense_reference(torch, w, dev, iters=3):
+    """Dense attention at the same B, H, N, D through torch's
+    scaled_dot_product_attention (library kernels, bf16), forward and
+    forward + backward: the comparison point for the sparse path.  Not part
+    of the LLSA path or of its timed region."""
+    import torch.nn.functional as F
+
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(4242)
+    shape = (w.B, w.H, w.N, w.D)
+    q, k, v = (torch.randn(shape, device=dev, dtype=dt, generator=gen).requires_grad_() for _ in range(3))
+    do = torch.randn(shape, device=dev, dtype=dt, generator=gen)
+
+    def timed(fn):
+        fn()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(iters):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / iters
+
+    with torch.no_grad():
+        fwd_ms = timed(lambda: F.scaled_dot_product_attention(q, k, v))
+
+    def fwd_bwd():
+        q.grad = k.grad = v.grad = None
+        F.scaled_dot_product_attention(q, k, v).backward(do)
+
+    fb_ms = timed(fwd_bwd)
+    del q, k, v, do
+    torch.cuda.empty_cache()
+    return {"impl": "torch.nn.functional.scaled_dot_product_attention (bf16, library kernels)",
+            "fwd_ms": round(fwd_ms, 3), "fwd_bwd_ms": round(fb_ms, 3), "iters": iters}
+
+
+def max_over_ranks(torch, dist, values, device) -> list:
+    """Element-wise maximum of per-rank timings (one all_reduce): the job's
+    time is its slowest rank's."""
+    t = torch.tensor([float(v) for v in values], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t.tolist()]
+
+
 def launches_per_step(L: int) -> dict:
     """Kernels each entry point launches (matches the C library's dispatch)."""
-    return {"pool": 1 + max(0, L - 2), "select": L, "fwd": 1, "transpose": 1,
+    return {"pool": 1 + max(0, L - 2), "select": L, "fwd": 1, "transpose": 4,
             "bwd": 2 + max(0, L - 1) + max(0, L - 2)}
 
 
@@ -263,7 +346,7 @@ def run_ours(args, rank, world, local_rank):
         if ev is not None:
             ev[3].record(stream)
         if w.backward:
-            llsa.llsa_index_transpose(desc, bufs.indices, bufs.csr, st, sh)
+            llsa.llsa_index_transpose(desc, bufs.indices, bufs.csr, bufs.tr_ws.data_ptr(), bufs.tr_ws_bytes, st, sh)
             if ev is not None:
                 ev[4].record(stream)
             dq, dk, dv = grads
@@ -335,9 +418,7 @@ def run_ours(args, rank, world, local_rank):
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
 
     if world > 1:
-        tt = torch.tensor([ms, e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms, e2e_ms = float(tt[0]), float(tt[1])
+        ms, e2e_ms = max_over_ranks(torch, dist, [ms, e2e_ms], dev)
     if int(bufs.status.item()) != 0:
         raise RuntimeError(f"device status {int(bufs.status.item())}")
     if rank != 0:
@@ -366,9 +447,20 @@ def run_ours(args, rank, world, local_rank):
         achieved = wk["bytes"] / (stage_ms[dom] * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s"}
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
+    roof["traffic"] = committed_traffic(args.workload, dom)
+    roof["traffic_source"] = (f"profiles/dram_traffic_{args.workload}.md (ncu dram__bytes_read.sum + "
+                              "dram__bytes_write.sum, summed over the call's launches)"
+                              if roof["traffic"] is not None else
+                              "null: no ncu capture of the current sources")
     roof["kernel"] = f"llsa_{'attn_' if dom in ('fwd', 'bwd') else ''}{dom} ({launches_per_step(w.L)[dom]} launches)"
     roof["peak_source"] = f"{peaks['source']} (MEASURED_PEAKS.json)" if peaks["source"] == "measured" else "fallback"
+    dense = None
+    if w.backward and not args.no_dense:
+        dense = dense_reference(torch, w, dev)
+        dense["llsa_fwd_ms"] = round(stage_ms["fwd"], 4)
+        dense["llsa_fwd_bwd_ms"] = round(stage_ms["fwd"] + stage_ms["bwd"], 4)
+        dense["speedup_fwd"] = round(dense["fwd_ms"] / stage_ms["fwd"], 2)
+        dense["speedup_fwd_bwd"] = round(dense["fwd_bwd_ms"] / dense["llsa_fwd_bwd_ms"], 2)
     attn_ms = stage_ms["fwd"] + stage_ms.get("bwd", 0.0)
     attn_flops = work["fwd"]["flops"] + (work["bwd"]["flops"] if w.backward else 0)
     sel_ms = stage_ms["pool"] + stage_ms["select"]
@@ -384,6 +476,7 @@ def run_ours(args, rank, world, local_rank):
         "selection_GBps": (work["pool"]["bytes"] + work["select"]["bytes"]) / (sel_ms * 1e-3) / 1e9,
         "roofline": roof,
         "cpu_baseline": cpu,
+        "dense_reference": dense,
         "e2e": {"value": world * tokens / (e2e_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": nlaunch * args.steps,
@@ -400,6 +493,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=workloads.HEADLINE, choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true",
+                    help="skip the dense scaled_dot_product_attention comparison")
     ap.add_argument("--fwd-tcgen05", action="store_true",
                     help="run the forward on the tcgen05 kernel (bf16, D=64)")
     args = ap.parse_args()

@@ -34,6 +34,7 @@ EXPORTED = (
     "llsa_pool",
     "llsa_select",
     "llsa_attn_fwd",
+    "llsa_transpose_workspace_bytes",
     "llsa_index_transpose",
     "llsa_bwd_workspace_bytes",
     "llsa_attn_bwd",
@@ -87,7 +88,9 @@ def lib() -> ctypes.CDLL:
             "llsa_select": (ctypes.c_int, [P(LlsaDesc), P(LlsaPyramid), P(LlsaIndices), vp]),
             "llsa_attn_fwd": (ctypes.c_int, [P(LlsaDesc), vp, vp, vp, P(LlsaPyramid), P(LlsaIndices),
                                              vp, vp, vp, vp]),
-            "llsa_index_transpose": (ctypes.c_int, [P(LlsaDesc), P(LlsaIndices), P(LlsaCsr), vp, vp]),
+            "llsa_transpose_workspace_bytes": (ctypes.c_size_t, [P(LlsaDesc)]),
+            "llsa_index_transpose": (ctypes.c_int, [P(LlsaDesc), P(LlsaIndices), P(LlsaCsr), vp,
+                                                    ctypes.c_size_t, vp, vp]),
             "llsa_bwd_workspace_bytes": (ctypes.c_size_t, [P(LlsaDesc)]),
             "llsa_attn_bwd": (ctypes.c_int, [P(LlsaDesc), vp, vp, vp, P(LlsaPyramid), vp, vp, vp,
                                              P(LlsaIndices), P(LlsaCsr), vp, vp, vp, vp, ctypes.c_size_t,
@@ -143,9 +146,13 @@ def llsa_attn_fwd(desc, q, k, v, pyramid, indices, o, lse, dev_status=None, stre
     return _check(st) if check else st
 
 
-def llsa_index_transpose(desc, indices, csr, dev_status=None, stream=0, check=True):
+def llsa_transpose_workspace_bytes(desc) -> int:
+    return int(lib().llsa_transpose_workspace_bytes(ctypes.byref(desc)))
+
+
+def llsa_index_transpose(desc, indices, csr, ws, ws_bytes, dev_status=None, stream=0, check=True):
     st = lib().llsa_index_transpose(ctypes.byref(desc), ctypes.byref(indices), ctypes.byref(csr),
-                                    dev_status, stream)
+                                    ws, ws_bytes, dev_status, stream)
     return _check(st) if check else st
 
 
@@ -213,6 +220,8 @@ class LlsaBuffers:
                 self.csr.col[l] = self.col[l].data_ptr()
         self.ws_bytes = llsa_bwd_workspace_bytes(desc) if with_bwd else 0
         self.ws = torch.empty(max(1, self.ws_bytes), dtype=torch.uint8, device=device)
+        self.tr_ws_bytes = llsa_transpose_workspace_bytes(desc) if with_bwd else 0
+        self.tr_ws = torch.empty(max(1, self.tr_ws_bytes), dtype=torch.uint8, device=device)
         self.status = torch.zeros(1, dtype=i32, device=device)
 
 

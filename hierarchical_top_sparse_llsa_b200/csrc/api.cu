@@ -53,6 +53,7 @@ struct WsLayout {
   size_t delta = 0;
   size_t part[kMaxL + 1] = {};
   size_t coarse[kMaxL + 1] = {};
+  size_t work = 0;
   size_t total = 0;
 };
 
@@ -70,6 +71,29 @@ inline WsLayout ws_layout(const llsa_desc* d) {
     w.part[l] = take(BH * (size_t)(d->N >> 7) * d->topk * 2 * d->D * sizeof(float));
   for (int l = 2; l <= d->L; ++l)
     w.coarse[l] = take(BH * (size_t)n_level(d, l) * 2 * d->D * sizeof(float));
+  w.work = take(sizeof(int32_t));
+  w.total = off;
+  return w;
+}
+
+// Transpose workspace: per level, BH * nchunk * N_l int32 counts.
+struct TrWsLayout {
+  size_t off[kMaxL + 1];
+  size_t total;
+};
+
+inline TrWsLayout tr_ws_layout(const llsa_desc* d) {
+  TrWsLayout w;
+  memset(&w, 0, sizeof(w));
+  size_t off = 0;
+  const size_t BH = (size_t)d->B * d->H;
+  for (int l = 1; l <= d->L; ++l) {
+    const int n = n_level(d, l);
+    int nchunk = 0, rows = 0;
+    transpose_chunking(n, &nchunk, &rows);
+    w.off[l] = off;
+    off += (BH * nchunk * n * sizeof(int32_t) + 255) & ~(size_t)255;
+  }
   w.total = off;
   return w;
 }
@@ -241,28 +265,42 @@ int llsa_attn_fwd(const llsa_desc* desc, const void* q, const void* k, const voi
   return launch_status(launch_attn_fwd_mma(p, maps, (cudaStream_t)stream));
 }
 
+size_t llsa_transpose_workspace_bytes(const llsa_desc* desc) {
+  if (check_desc(desc) != LLSA_OK) return 0;
+  return tr_ws_layout(desc).total;
+}
+
 int llsa_index_transpose(const llsa_desc* desc, const llsa_indices* idx, const llsa_csr* out,
-                         int32_t* dev_status, void* stream) {
+                         void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
   int st = check_desc(desc);
   if (st != LLSA_OK) return st;
-  if (idx == nullptr || out == nullptr || !indices_present(desc, idx)) return LLSA_ERR_INVALID_ARG;
+  if (idx == nullptr || out == nullptr || ws == nullptr || !indices_present(desc, idx))
+    return LLSA_ERR_INVALID_ARG;
+  if (((uintptr_t)ws & 255) != 0) return LLSA_ERR_INVALID_ARG;
+  const TrWsLayout w = tr_ws_layout(desc);
+  if (ws_bytes < w.total) return LLSA_ERR_WORKSPACE;
   TransposeParams p;
   memset(&p, 0, sizeof(p));
   p.BH = desc->B * desc->H;
   p.K = desc->topk;
   p.status = dev_status;
   p.nlev = desc->L;
-  int cta = 0;
+  int cta = 0, tile = 0, scan = 0;
   for (int l = 1; l <= desc->L; ++l) {
     if (out->row_ptr[l] == nullptr || out->col[l] == nullptr) return LLSA_ERR_INVALID_ARG;
     TransposeLevel& t = p.lv[l - 1];
     t.idx = idx->idx[l];
     t.row_ptr = out->row_ptr[l];
     t.col = out->col[l];
+    t.cnt = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + w.off[l]);
     t.n = n_level(desc, l);
-    t.ranges = (t.n + 255) / 256;
+    transpose_chunking(t.n, &t.nchunk, &t.rows);
     t.cta_begin = cta;
-    cta += p.BH * t.ranges;
+    t.tile_begin = tile;
+    t.scan_begin = scan;
+    cta += p.BH * t.nchunk;
+    tile += p.BH * transpose_prefix_tiles(t.n);
+    scan += p.BH;
   }
   return launch_status(launch_transpose(p, (cudaStream_t)stream));
 }
@@ -303,6 +341,7 @@ int llsa_attn_bwd(const llsa_desc* desc, const void* q, const void* k, const voi
     p.part[l] = reinterpret_cast<float*>(base + w.part[l]);
     p.coarse[l] = reinterpret_cast<float*>(base + w.coarse[l]);
   }
+  p.work = reinterpret_cast<int32_t*>(base + w.work);
   p.dq = dq;
   p.dk = dk;
   p.dv = dv;

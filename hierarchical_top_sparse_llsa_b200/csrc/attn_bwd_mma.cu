@@ -28,6 +28,8 @@
 
 #include <math.h>
 
+#include <algorithm>
+
 #include "keyset.cuh"
 #include "mma_tiles.cuh"
 
@@ -36,16 +38,8 @@ namespace llsa {
 namespace {
 
 constexpr int kQWarps = 8;   // query blocks per CTA in pass 1 (one partial group)
-constexpr int kKVWarps = 4;  // key blocks per CTA in pass 3
 constexpr int kRing = 2;
 constexpr float kLog2e = 1.4426950408889634f;
-
-__device__ __forceinline__ void zero_acc(float (&s)[2][4]) {
-#pragma unroll
-  for (int a = 0; a < 2; ++a)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) s[a][e] = 0.f;
-}
 
 // P = exp2(S * sc2 + lw - lse2) on a 16x16 tile (rows g, g+8 of the query
 // side); rows with lse = -inf get P = 0.
@@ -105,6 +99,7 @@ bwd_q_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
   const int g = lane >> 2, t = lane & 3;
   const int bh = blockIdx.y;
   const int grp = blockIdx.x;
+  if (grp == 0 && bh == 0 && threadIdx.x == 0) *p.work = 0;  // pass 3's work counter
   const int n1 = p.N >> 4;
   const int b = grp * kQWarps + warp;
   const bool active = b < n1;
@@ -424,168 +419,231 @@ bwd_q_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
 }
 
 template <int D>
-__global__ void __launch_bounds__(kKVWarps * 32)
+__global__ void __launch_bounds__(32)
 bwd_kv_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                   const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
                   AttnParams p) {
   constexpr int TILE = 32 * D;
   constexpr int NT = D / 8;
   constexpr int HALVES = D / 64;
-  constexpr int SIDE = 128;  // LSE[16] and Delta[16] of a stage's query block (fp32)
-  // per warp: K_c | V_c | kRing x (Q | dO) tiles, then kRing side buffers; every
-  // tile stays 1024-byte aligned for the 128-byte swizzle
-  constexpr int WARP_BYTES = 2 * TILE * (1 + kRing) + 1024;
+  constexpr int SIDE = 128;       // LSE[16] and Delta[16] of a stage's query block (fp32)
+  constexpr int CROW = 2 * D * 4;  // one coarse gradient row dK(l) | dV(l), fp32
+  // K_c | V_c | kRing x (Q | dO) tiles (each 1024-byte aligned for the
+  // 128-byte swizzle), kRing side buffers, two sets of L-1 coarse rows
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  __shared__ __align__(8) uint64_t bars_all[kKVWarps][1 + kRing];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ __align__(8) uint64_t bars[1 + kRing];  // [0]: K/V + coarse rows; then the ring
+  const int lane = threadIdx.x;
   const int g = lane >> 2, t = lane & 3;
-  const int bh = blockIdx.y;
   const int n1 = p.N >> 4;
-  const int c = blockIdx.x * kKVWarps + warp;  // key block
-  const bool active = c < n1;
-  const int K = p.K;
+  const int items = p.B * p.H * n1;
+  const int K = p.K, L = p.L;
 
-  unsigned char* wb = sm + (size_t)warp * WARP_BYTES;
-  const uint32_t w0 = smem_u32(wb);
+  const uint32_t w0 = smem_u32(sm);
   const uint32_t kt = w0, vt = w0 + TILE;
   auto ring_q = [&](int st) { return w0 + (uint32_t)(2 + 2 * st) * TILE; };
   auto ring_do = [&](int st) { return w0 + (uint32_t)(3 + 2 * st) * TILE; };
-  const uint32_t side0 = w0 + (uint32_t)(2 + 2 * kRing) * TILE;
-  auto side_of = [&](int st) {
-    return reinterpret_cast<const float*>(wb + (2 + 2 * kRing) * TILE + st * SIDE);
-  };
-  const uint32_t bar0 = smem_u32(&bars_all[warp][0]);
-  auto bar_of = [&](int st) { return bar0 + 8u * (1 + st); };
+  unsigned char* sideb = sm + (2 + 2 * kRing) * TILE;
+  const uint32_t side0 = smem_u32(sideb);
+  unsigned char* cgb = sideb + kRing * SIDE;
+  const uint32_t kvbar = smem_u32(&bars[0]);
+  auto bar_of = [&](uint32_t pos) { return smem_u32(&bars[1 + pos % kRing]); };
+  auto par_of = [&](uint32_t pos) { return (pos / kRing) & 1u; };
   if (lane == 0) {
-    for (int i = 0; i <= kRing; ++i) mbar_init(bar0 + 8u * i, 1);
+    for (int i = 0; i <= kRing; ++i) mbar_init(smem_u32(&bars[i]), 1);
     fence_mbar_init();
   }
   __syncwarp();
-  if (!active) return;
 
-  const size_t rowbase = (size_t)bh * p.N;
-  const int32_t* rp = p.row_ptr[1] + (size_t)bh * (n1 + 1);
-  const int32_t* col = p.col[1] + (size_t)bh * n1 * K;
-  const int beg = rp[c];
-  const int nq = rp[c + 1] - beg;
-  auto issue = [&](int r) {
+  // One key block's row of the level-1 key-major lists.  colw holds
+  // col[beg + 32 * win + lane], a window of the row's query blocks.
+  struct Row {
+    int item, bh, c, beg, nq, colw, win;
+  };
+  auto row_bounds = [&](int item, Row& R) {
+    R.item = item;
+    R.bh = 0, R.c = 0, R.beg = 0, R.nq = 0, R.colw = 0, R.win = -1;
+    if (item < items) {
+      R.bh = item / n1;
+      R.c = item - R.bh * n1;
+      const int32_t* rp = p.row_ptr[1] + (size_t)R.bh * (n1 + 1);
+      R.beg = rp[R.c];
+      R.nq = rp[R.c + 1] - R.beg;
+    }
+  };
+  auto row_window = [&](Row& R, int win) {
+    R.win = win;
+    const int j = 32 * win + lane;
+    R.colw = (j < R.nq) ? p.col[1][(size_t)R.bh * n1 * K + R.beg + j] : 0;
+  };
+  // ring position pos <- tile r of row R (all lanes call; lane 0 issues)
+  auto issue = [&](Row& R, int r, uint32_t pos) {
+    if ((r >> 5) != R.win) row_window(R, r >> 5);
+    const int qb = __shfl_sync(0xffffffffu, R.colw, r & 31);
     if (lane == 0) {
-      const int qb = col[beg + r];
-      const int st = r % kRing;
-      mbar_arrive_expect_tx(bar_of(st), 2u * TILE + SIDE);
-      const size_t row0 = rowbase + (size_t)qb * 16;
+      const uint32_t st = pos % kRing;
+      const uint32_t bar = bar_of(pos);
+      mbar_arrive_expect_tx(bar, 2u * TILE + SIDE);
+      const size_t row0 = (size_t)R.bh * p.N + (size_t)qb * 16;
       const int y = (int)row0;
 #pragma unroll
       for (int h = 0; h < HALVES; ++h) {
-        tma_load_2d(ring_q(st) + h * 2048, &tq, 64 * h, y, bar_of(st));
-        tma_load_2d(ring_do(st) + h * 2048, &tdo, 64 * h, y, bar_of(st));
+        tma_load_2d(ring_q(st) + h * 2048, &tq, 64 * h, y, bar);
+        tma_load_2d(ring_do(st) + h * 2048, &tdo, 64 * h, y, bar);
       }
-      bulk_load(side0 + st * SIDE, p.lse_in + row0, 64, bar_of(st));
-      bulk_load(side0 + st * SIDE + 64, p.delta + row0, 64, bar_of(st));
+      bulk_load(side0 + st * SIDE, p.lse_in + row0, 64, bar);
+      bulk_load(side0 + st * SIDE + 64, p.delta + row0, 64, bar);
     }
   };
-  if (lane == 0) {
-    mbar_arrive_expect_tx(bar0, 2u * TILE);
-    const int y = (int)(rowbase + (size_t)c * 16);
+  // K_c, V_c (if the row is not empty) and the coarse gradient rows of key
+  // block c into coarse buffer `par`
+  auto issue_kv = [&](const Row& R, int par) {
+    if (lane == 0) {
+      const uint32_t bytes = (R.nq > 0 ? 2u * TILE : 0u) + (uint32_t)(L - 1) * CROW;
+      mbar_arrive_expect_tx(kvbar, bytes);
+      if (R.nq > 0) {
+        const int y = (int)((size_t)R.bh * p.N + (size_t)R.c * 16);
 #pragma unroll
-    for (int h = 0; h < HALVES; ++h) {
-      tma_load_2d(kt + h * 2048, &tk, 64 * h, y, bar0);
-      tma_load_2d(vt + h * 2048, &tv, 64 * h, y, bar0);
+        for (int h = 0; h < HALVES; ++h) {
+          tma_load_2d(kt + h * 2048, &tk, 64 * h, y, kvbar);
+          tma_load_2d(vt + h * 2048, &tv, 64 * h, y, kvbar);
+        }
+      }
+      for (int l = 2; l <= L; ++l) {
+        const size_t tc = (size_t)R.bh * (p.N >> (4 * l)) + (R.c >> (4 * (l - 1)));
+        bulk_load(smem_u32(cgb + (size_t)(par * (L - 1) + (l - 2)) * CROW), p.coarse[l] + tc * 2 * D, CROW,
+                  kvbar);
+      }
     }
-  }
-  for (int r = 0; r < nq && r < kRing; ++r) issue(r);
+  };
 
-  bool ok = mbar_wait_bounded(bar0, 0);
-  float dk[NT][4], dv[NT][4];
-#pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    dk[nt][0] = dk[nt][1] = dk[nt][2] = dk[nt][3] = 0.f;
-    dv[nt][0] = dv[nt][1] = dv[nt][2] = dv[nt][3] = 0.f;
+  // work items are key blocks, taken in order from a counter that pass 1 zeroed
+  int nxt_l0 = (lane == 0) ? atomicAdd(p.work, 1) : 0;
+  Row cur;
+  row_bounds(__shfl_sync(0xffffffffu, nxt_l0, 0), cur);
+  nxt_l0 = (lane == 0) ? atomicAdd(p.work, 1) : 0;
+  uint32_t pos = 0;     // ring position of cur's first tile
+  uint32_t issued = 0;  // ring positions issued so far
+  uint32_t kvph = 0;
+  int par = 0;
+  bool kv_pending = false;
+  if (cur.item < items) {
+    issue_kv(cur, par);
+    kv_pending = true;
+    for (int r = 0; r < cur.nq && r < kRing; ++r) issue(cur, r, issued++);
   }
   const float sc2 = p.scale * kLog2e;
-  // software pipeline: S^T and dP^T of query block r+1 are issued before the
-  // elementwise step and the dV/dK products of block r
-  float s_cur[2][4], d_cur[2][4];
-  int r = 0;
-  if (nq > 0 && ok) {
-    ok = mbar_wait_bounded(bar_of(0), 0);
-    if (ok) {
-      qk_tile_ss<D>(kt, ring_q(0), lane, s_cur);
-      qk_tile_ss<D>(vt, ring_do(0), lane, d_cur);
-    }
-  }
-  for (; r < nq && ok; ++r) {
-    const int st = r % kRing;
-    float s_nx[2][4], d_nx[2][4];
-    if (r + 1 < nq) {
-      const int ns = (r + 1) % kRing;
-      ok = mbar_wait_bounded(bar_of(ns), (uint32_t)(((r + 1) / kRing) & 1));
-      if (!ok) break;
-      qk_tile_ss<D>(kt, ring_q(ns), lane, s_nx);
-      qk_tile_ss<D>(vt, ring_do(ns), lane, d_nx);
-    }
-    // LSE and Delta of the queries in this thread's columns: 2t, 2t+1, 8+2t, 9+2t
-    const float* side = side_of(st);
-    float P[2][4], dS[2][4];
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int qi = 8 * nt + 2 * t + (e & 1);
-        const float l2 = side[qi] * kLog2e;
-        P[nt][e] = (l2 == -INFINITY) ? 0.f : ex2_approx(fmaf(s_cur[nt][e], sc2, -l2));
-        dS[nt][e] = P[nt][e] * (d_cur[nt][e] - side[16 + qi]);
-      }
-    uint32_t ph[4], pl[4], dsh[4], dsl[4];
-    split_frag(P, ph, pl);
-    split_frag(dS, dsh, dsl);
-    pv_tile2<D>(ph, pl, ring_do(st), lane, dv);
-    pv_tile2<D>(dsh, dsl, ring_q(st), lane, dk);
-    __syncwarp();
-    fence_proxy_async_smem();
-    if (r + kRing < nq) issue(r + kRing);
-    if (r + 1 < nq) {
-#pragma unroll
-      for (int a = 0; a < 2; ++a)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          s_cur[a][e] = s_nx[a][e];
-          d_cur[a][e] = d_nx[a][e];
-        }
-    }
-  }
-  if (!ok) {
-    for (int q = r; q < nq && q < r + kRing; ++q)
-      mbar_wait_bounded(bar_of(q % kRing), (uint32_t)((q / kRing) & 1));
-    if (lane == 0) report_status(p.status, LLSA_DEV_TIMEOUT);
-    return;
-  }
-  // epilogue: dK = scale * acc + sum_l coarse dK(l)[t >> 4l] / 16^l (likewise dV)
-  bf16* dK = static_cast<bf16*>(p.dk);
-  bf16* dV = static_cast<bf16*>(p.dv);
-#pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const size_t tok = (size_t)c * 16 + g + 8 * half;
+  bool ok = true;
+  while (cur.item < items && ok) {
+    Row nxt;
+    row_bounds(__shfl_sync(0xffffffffu, nxt_l0, 0), nxt);  // loads stay in flight
+    nxt_l0 = (lane == 0) ? atomicAdd(p.work, 1) : 0;         // likewise
+    ok = mbar_wait_bounded(kvbar, kvph);
+    if (!ok) break;
+    kv_pending = false;
+    kvph ^= 1u;
+
+    float dk[NT][4], dv[NT][4];
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      const int d = 8 * nt + 2 * t;
-      float k0 = dk[nt][2 * half] * p.scale, k1 = dk[nt][2 * half + 1] * p.scale;
-      float v0 = dv[nt][2 * half], v1 = dv[nt][2 * half + 1];
-      for (int l = 2; l <= p.L; ++l) {
-        const float inv = 1.0f / (float)(1u << (4 * l));
-        const float* cg = p.coarse[l] + ((size_t)bh * (p.N >> (4 * l)) + (tok >> (4 * l))) * 2 * D;
-        const float2 gk = *reinterpret_cast<const float2*>(cg + d);
-        const float2 gv = *reinterpret_cast<const float2*>(cg + D + d);
-        k0 += gk.x * inv;
-        k1 += gk.y * inv;
-        v0 += gv.x * inv;
-        v1 += gv.y * inv;
-      }
-      *reinterpret_cast<uint32_t*>(dK + (rowbase + tok) * D + d) = pack_bf16(k0, k1);
-      *reinterpret_cast<uint32_t*>(dV + (rowbase + tok) * D + d) = pack_bf16(v0, v1);
+      dk[nt][0] = dk[nt][1] = dk[nt][2] = dk[nt][3] = 0.f;
+      dv[nt][0] = dv[nt][1] = dv[nt][2] = dv[nt][3] = 0.f;
     }
+    const int nq = cur.nq;
+    // software pipeline: S^T and dP^T of query block r+1 are issued before
+    // the elementwise step and the dV/dK products of block r
+    float s_cur[2][4], d_cur[2][4];
+    if (nq > 0) {
+      ok = mbar_wait_bounded(bar_of(pos), par_of(pos));
+      if (!ok) break;
+      qk_tile_ss<D>(kt, ring_q(pos % kRing), lane, s_cur);
+      qk_tile_ss<D>(vt, ring_do(pos % kRing), lane, d_cur);
+    }
+    if (nxt.item < items) row_window(nxt, 0);  // its query blocks, for the first issues below
+    for (int r = 0; r < nq; ++r) {
+      const uint32_t pr = pos + r;
+      float s_nx[2][4], d_nx[2][4];
+      if (r + 1 < nq) {
+        ok = mbar_wait_bounded(bar_of(pr + 1), par_of(pr + 1));
+        if (!ok) break;
+        qk_tile_ss<D>(kt, ring_q((pr + 1) % kRing), lane, s_nx);
+        qk_tile_ss<D>(vt, ring_do((pr + 1) % kRing), lane, d_nx);
+      }
+      // LSE and Delta of the queries in this thread's columns: 2t, 2t+1, 8+2t, 9+2t
+      const float* side = reinterpret_cast<const float*>(sideb + (pr % kRing) * SIDE);
+      float P[2][4], dS[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int qi = 8 * nt + 2 * t + (e & 1);
+          const float l2 = side[qi] * kLog2e;
+          P[nt][e] = (l2 == -INFINITY) ? 0.f : ex2_approx(fmaf(s_cur[nt][e], sc2, -l2));
+          dS[nt][e] = P[nt][e] * (d_cur[nt][e] - side[16 + qi]);
+        }
+      uint32_t ph[4], pl[4], dsh[4], dsl[4];
+      split_frag(P, ph, pl);
+      split_frag(dS, dsh, dsl);
+      pv_tile2<D>(ph, pl, ring_do(pr % kRing), lane, dv);
+      pv_tile2<D>(dsh, dsl, ring_q(pr % kRing), lane, dk);
+      __syncwarp();
+      fence_proxy_async_smem();
+      if (r + kRing < nq) issue(cur, r + kRing, issued++);
+      if (r + 1 < nq) {
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            s_cur[a][e] = s_nx[a][e];
+            d_cur[a][e] = d_nx[a][e];
+          }
+      }
+    }
+    if (!ok) break;
+    pos += nq;
+    // the next row's loads go out before this row's epilogue
+    __syncwarp();
+    fence_proxy_async_smem();
+    if (nxt.item < items) {
+      issue_kv(nxt, par ^ 1);
+      kv_pending = true;
+      for (int r = 0; r < nxt.nq && r < kRing; ++r) issue(nxt, r, issued++);
+    }
+    // epilogue: dK = scale * acc + sum_l coarse dK(l)[t >> 4l] / 16^l (likewise dV)
+    bf16* dK = static_cast<bf16*>(p.dk);
+    bf16* dV = static_cast<bf16*>(p.dv);
+    const size_t rowbase = (size_t)cur.bh * p.N;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const size_t tok = (size_t)cur.c * 16 + g + 8 * half;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int d = 8 * nt + 2 * t;
+        float k0 = dk[nt][2 * half] * p.scale, k1 = dk[nt][2 * half + 1] * p.scale;
+        float v0 = dv[nt][2 * half], v1 = dv[nt][2 * half + 1];
+        for (int l = 2; l <= L; ++l) {
+          const float inv = 1.0f / (float)(1u << (4 * l));
+          const float* cg = reinterpret_cast<const float*>(cgb + (size_t)(par * (L - 1) + (l - 2)) * CROW);
+          const float2 gk = *reinterpret_cast<const float2*>(cg + d);
+          const float2 gv = *reinterpret_cast<const float2*>(cg + D + d);
+          k0 += gk.x * inv;
+          k1 += gk.y * inv;
+          v0 += gv.x * inv;
+          v1 += gv.y * inv;
+        }
+        *reinterpret_cast<uint32_t*>(dK + (rowbase + tok) * D + d) = pack_bf16(k0, k1);
+        *reinterpret_cast<uint32_t*>(dV + (rowbase + tok) * D + d) = pack_bf16(v0, v1);
+      }
+    }
+    cur = nxt;
+    par ^= 1;
+  }
+  if (!ok) {
+    // let every copy still in flight land before the CTA exits
+    if (kv_pending) mbar_wait_bounded(kvbar, kvph);
+    for (uint32_t q = pos; q < issued; ++q) mbar_wait_bounded(bar_of(q), par_of(q));
+    if (lane == 0) report_status(p.status, LLSA_DEV_TIMEOUT);
   }
 }
 
@@ -607,12 +665,19 @@ cudaError_t launch_typed(const AttnParams& p, const CUtensorMap* maps, cudaStrea
   // pass 2
   e = launch_coarse_reduce(p, s);
   if (e != cudaSuccess) return e;
-  // pass 3
-  const size_t smem3 = 1024 + (size_t)kKVWarps * (2 * TILE * (1 + kRing) + 1024);
+  // pass 3: persistent single-warp CTAs, as many as fit at once
+  const size_t smem3 = 1024 + (size_t)2 * TILE * (1 + kRing) + kRing * 128 +
+                       (size_t)2 * (p.L - 1) * 2 * D * sizeof(float);
   e = cudaFuncSetAttribute(bwd_kv_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3);
   if (e != cudaSuccess) return e;
-  bwd_kv_mma_kernel<D><<<dim3((n1 + kKVWarps - 1) / kKVWarps, BH), kKVWarps * 32, smem3, s>>>(
-      maps[0], maps[1], maps[2], maps[3], p);
+  int dev = 0, nsm = 0, per_sm = 0;
+  e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, bwd_kv_mma_kernel<D>, 32, smem3);
+  if (e != cudaSuccess) return e;
+  const long items = (long)BH * n1;
+  const int grid3 = (int)std::min<long>(items, (long)nsm * std::max(per_sm, 1));
+  bwd_kv_mma_kernel<D><<<grid3, 32, smem3, s>>>(maps[0], maps[1], maps[2], maps[3], p);
   return cudaGetLastError();
 }
 

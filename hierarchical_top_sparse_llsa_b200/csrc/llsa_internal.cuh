@@ -79,13 +79,14 @@ struct RowRule {
 // for lanes outside every row (their results are ignored and they are never
 // read by lanes inside a row).  Segmented shuffle scans give, for each entry,
 // the largest in-range entry before it and whether a pad came before it.
-// Must be called by all 32 lanes.
-__device__ __forceinline__ bool warp_row_used(int v, int slot, int n, bool on, int& flags) {
+// Must be called by all 32 lanes; seg, the same on every lane, is at least
+// the row length (the scans stop once they span that many slots).
+__device__ __forceinline__ bool warp_row_used(int v, int slot, int n, bool on, int& flags, int seg = 32) {
   const bool inr = on && v >= 0 && v < n;
   int mx = inr ? v : -1;
   int pad = (on && v == -1) ? 1 : 0;
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
+  for (int o = 1; o < seg; o <<= 1) {
     const int y = __shfl_up_sync(0xffffffffu, mx, o);
     const int z = __shfl_up_sync(0xffffffffu, pad, o);
     if (slot >= o) {
@@ -132,9 +133,13 @@ struct TransposeLevel {
   const int32_t* idx;
   int32_t* row_ptr;
   int32_t* col;
-  int n;          // N_l (queries == keys at level l)
-  int cta_begin;  // first CTA of this level in the grid
-  int ranges;     // key ranges per (b, h)
+  int32_t* cnt;    // workspace [BH][nchunk][n]: per-chunk key counts, then cursors
+  int n;           // N_l (queries == keys at level l)
+  int nchunk;      // row chunks per (b, h)
+  int rows;        // rows per chunk
+  int cta_begin;   // first CTA of this level in the count and fill grids
+  int tile_begin;  // first CTA of this level in the chunk-prefix grid
+  int scan_begin;  // first CTA of this level in the row_ptr scan grid
 };
 
 struct TransposeParams {
@@ -165,6 +170,7 @@ struct AttnParams {
   float* delta;                 // [BH, N]
   float* part[kMaxL + 1];       // [BH, N/128, K, 2, D] per coarse level (groups of 8 query blocks)
   float* coarse[kMaxL + 1];     // [BH, N_l, 2, D] per coarse level
+  int32_t* work;                // pass-3 work counter (zeroed by pass 1)
   int32_t* status;
   int B, H, N, D, L, K;
   float scale;
@@ -175,6 +181,8 @@ struct AttnParams {
 cudaError_t launch_pool(const PoolParams& p, int dtype, cudaStream_t s);
 cudaError_t launch_select_level(const SelectParams& p, int BH, int D, cudaStream_t s);
 cudaError_t launch_transpose(const TransposeParams& p, cudaStream_t s);
+void transpose_chunking(int n, int* nchunk, int* rows);
+int transpose_prefix_tiles(int n);
 cudaError_t launch_coarse_reduce(const AttnParams& p, cudaStream_t s);
 
 }  // namespace llsa

@@ -1,21 +1,27 @@
 // Sparse index transpose (Step 4 of the howistudyai explainer of "Trainable
 // Log-linear Sparse Attention for Efficient Diffusion Transformers";
 // Building Blocks: Sparse Index Transpose): query-major index lists I(l) to
-// key-major CSR lists, by counting, prefix-summing and filling, with no dense
-// mask and no global atomics.
+// key-major CSR lists, with no dense mask and no global atomics.
 //
-// One launch covers every level.  A CTA owns (level, b*h, a range of 256 key
-// tokens) and walks all index rows of its (level, b, h) twice:
-//   pass 1 counts, per warp, the used entries that fall in its key range
-//          (warp-private shared-memory histograms) and those below it;
-//   scan   turns the counts into row offsets: keys below the range come
-//          first, then an exclusive scan over the range, then per-warp bases;
-//   pass 2 writes each query token at its key's cursor.  Warps own
-//          contiguous query slices in order, rows are walked in order inside
-//          a warp, and lanes that share a key in one step are ranked by
-//          __match_any_sync, so each key's list comes out ascending.
-// The whole result is deterministic.  Entries are screened with the same
-// used-entry rule as the attention kernels.
+// A stable counting sort of the (key, query) pairs by key, in four launches
+// that each cover every level.  The query rows of a (level, b, h) are cut
+// into nchunk chunks of consecutive rows; the workspace holds one count per
+// (chunk, key).
+//   count   one CTA per chunk: shared-memory histogram of the chunk's used
+//           entries, written out as that chunk's row of counts;
+//   prefix  one CTA per 1024 keys: per key, the running sum over chunks (in
+//           place: each count becomes the chunk's first slot relative to the
+//           key's list) and the key's total, parked in row_ptr;
+//   scan    one CTA per (level, b, h): the exclusive scan of the totals into
+//           row_ptr, and -1 in the unused tail of col;
+//   fill    one CTA per chunk: the cursors row_ptr[c] + first slot are staged
+//           in shared memory, then one warp walks the chunk's rows in order,
+//           lanes that share a key in one step ranked by __match_any_sync,
+//           and writes each query at its key's cursor.
+// Chunks are filled in row order from the slots the prefix gave them, so
+// every key's list comes out ascending and the result is deterministic.
+// Entries are screened with the same used-entry rule as the attention
+// kernels; the count launch reports the status bits.
 
 #include "llsa_internal.cuh"
 
@@ -23,147 +29,280 @@ namespace llsa {
 
 namespace {
 
-constexpr int kTrWarps = 16;
-constexpr int kTrRange = 256;
-constexpr int kBatch = 8;  // row steps whose index loads are in flight together
+constexpr int kCountThreads = 256;
+constexpr int kPrefixThreads = 256;
+constexpr int kPrefixKeys = 4 * kPrefixThreads;  // keys per prefix CTA
+constexpr int kScanThreads = 1024;
+constexpr int kFillThreads = 256;  // all stage the cursors; warp 0 fills
+constexpr int kMaxChunks = 32;     // row chunks per (level, b, h); see transpose_chunking
+constexpr int kRangeKeys = 8192;   // keys per shared-memory histogram / cursor range
+constexpr int kBatch = 8;          // row steps whose index loads are in flight together
 
-__global__ void __launch_bounds__(kTrWarps * 32)
-transpose_kernel(TransposeParams p) {
-  __shared__ int hist[kTrWarps][kTrRange];
-  __shared__ int below[kTrWarps];
-  __shared__ int scan_buf[kTrRange];
-  __shared__ int below_total;
+enum Grid { kChunkGrid, kTileGrid, kScanGrid };
 
-  // which level this CTA works on
+__device__ __forceinline__ int grid_begin(const TransposeLevel& t, Grid g) {
+  return g == kChunkGrid ? t.cta_begin : (g == kTileGrid ? t.tile_begin : t.scan_begin);
+}
+
+__device__ __forceinline__ int level_of(const TransposeParams& p, int blk, Grid g) {
   int lvl = 0;
-  while (lvl + 1 < p.nlev && (int)blockIdx.x >= p.lv[lvl + 1].cta_begin) ++lvl;
-  const TransposeLevel L = p.lv[lvl];
-  const int local = blockIdx.x - L.cta_begin;
-  const int bh = local / L.ranges;
-  const int c0 = (local % L.ranges) * kTrRange;
-  const int c1 = min(L.n, c0 + kTrRange);
-  const int K = p.K;
-  const int n = L.n;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  while (lvl + 1 < p.nlev && blk >= grid_begin(p.lv[lvl + 1], g)) ++lvl;
+  return lvl;
+}
 
+// How one warp lays index rows across its lanes: rows_per_step rows of K
+// slots side by side; lanes past the last full row stay idle.
+struct RowLanes {
+  int rows_per_step, sub, slot;
+  bool on;
+  __device__ __forceinline__ RowLanes(int K, int lane) {
+    rows_per_step = 32 / K;  // K <= 32
+    sub = lane / K;
+    on = sub < rows_per_step;
+    slot = on ? lane % K : lane;  // idle lanes never feed a row
+  }
+};
+
+__global__ void __launch_bounds__(kCountThreads)
+tr_count_kernel(TransposeParams p) {
+  __shared__ int hist[kRangeKeys];
+  const TransposeLevel L = p.lv[level_of(p, blockIdx.x, kChunkGrid)];
+  const int local = blockIdx.x - L.cta_begin;
+  const int bh = local / L.nchunk, ch = local % L.nchunk;
+  const int n = L.n, K = p.K;
+  const int r0 = ch * L.rows, r1 = min(n, r0 + L.rows);
   const int32_t* I = L.idx + (size_t)bh * n * K;
+  int32_t* cnt = L.cnt + ((size_t)bh * L.nchunk + ch) * n;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const RowLanes rl(K, lane);
+  const int stride = (kCountThreads / 32) * rl.rows_per_step * kBatch;
+
+  int flags = 0;
+  for (int k0 = 0; k0 < n; k0 += kRangeKeys) {
+    const int k1 = min(n, k0 + kRangeKeys);
+    for (int e = threadIdx.x; e < k1 - k0; e += blockDim.x) hist[e] = 0;
+    __syncthreads();
+    for (int rb = r0 + warp * rl.rows_per_step * kBatch; rb < r1; rb += stride) {
+      int cb[kBatch];
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        const int q = rb + i * rl.rows_per_step + rl.sub;
+        cb[i] = (rl.on && q < r1) ? I[(size_t)q * K + rl.slot] : -1;
+      }
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        const int q = rb + i * rl.rows_per_step + rl.sub;
+        const int c = cb[i];
+        const bool u = warp_row_used(c, rl.slot, n, rl.on && q < r1, flags, K);
+        if (u && c >= k0 && c < k1) atomicAdd(&hist[c - k0], 1);
+      }
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < k1 - k0; e += blockDim.x) cnt[k0 + e] = hist[e];
+    __syncthreads();
+  }
+  flags = __reduce_or_sync(0xffffffffu, flags);
+  if (lane == 0) report_status(p.status, flags);
+}
+
+__global__ void __launch_bounds__(kPrefixThreads)
+tr_prefix_kernel(TransposeParams p) {
+  const TransposeLevel L = p.lv[level_of(p, blockIdx.x, kTileGrid)];
+  const int n = L.n, nch = L.nchunk;
+  const int tiles = (n + kPrefixKeys - 1) / kPrefixKeys;
+  const int local = blockIdx.x - L.tile_begin;
+  const int bh = local / tiles;
+  const int c0 = (local % tiles) * kPrefixKeys + 4 * threadIdx.x;
+  if (c0 >= n) return;
+  int32_t* cnt = L.cnt + (size_t)bh * nch * n;
+  int32_t* tot = L.row_ptr + (size_t)bh * (n + 1);
+  if ((n & 3) == 0) {
+    // four keys per thread as one int4; 8 chunks' loads in flight at a time
+    int4 run = make_int4(0, 0, 0, 0);
+    for (int ch0 = 0; ch0 < nch; ch0 += 8) {
+      int4 v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (ch0 + i < nch) v[i] = *reinterpret_cast<const int4*>(cnt + (size_t)(ch0 + i) * n + c0);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        if (ch0 + i < nch) {
+          *reinterpret_cast<int4*>(cnt + (size_t)(ch0 + i) * n + c0) = run;
+          run.x += v[i].x;
+          run.y += v[i].y;
+          run.z += v[i].z;
+          run.w += v[i].w;
+        }
+      }
+    }
+    tot[c0] = run.x;
+    tot[c0 + 1] = run.y;
+    tot[c0 + 2] = run.z;
+    tot[c0 + 3] = run.w;
+  } else {
+    for (int j = 0; j < 4 && c0 + j < n; ++j) {
+      int run = 0;
+      for (int ch = 0; ch < nch; ++ch) {
+        int32_t* a = cnt + (size_t)ch * n + c0 + j;
+        const int v = *a;
+        *a = run;
+        run += v;
+      }
+      tot[c0 + j] = run;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kScanThreads)
+tr_scan_kernel(TransposeParams p) {
+  __shared__ int warp_tot[kScanThreads / 32];
+  const TransposeLevel L = p.lv[level_of(p, blockIdx.x, kScanGrid)];
+  const int bh = blockIdx.x - L.scan_begin;
+  const int n = L.n, K = p.K;
   int32_t* row_ptr = L.row_ptr + (size_t)bh * (n + 1);
   int32_t* col = L.col + (size_t)bh * n * K;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  for (int e = threadIdx.x; e < kTrWarps * kTrRange; e += blockDim.x) (&hist[0][0])[e] = 0;
-  __syncthreads();
+  int carry = 0;  // entries of the keys before this tile
+  for (int t0 = 0; t0 < n; t0 += 4 * kScanThreads) {
+    const int c0 = t0 + 4 * threadIdx.x;
+    int tot[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) tot[j] = (c0 + j < n) ? row_ptr[c0 + j] : 0;
+    const int mine = tot[0] + tot[1] + tot[2] + tot[3];
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) warp_tot[warp] = incl;
+    __syncthreads();
+    int before = 0, tile_total = 0;
+    for (int w = 0; w < kScanThreads / 32; ++w) {
+      const int x = warp_tot[w];
+      if (w < warp) before += x;
+      tile_total += x;
+    }
+    int run = carry + before + incl - mine;  // first slot of key c0
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (c0 + j < n) row_ptr[c0 + j] = run;
+      run += tot[j];
+    }
+    carry += tile_total;
+    __syncthreads();  // warp_tot is rewritten by the next tile
+  }
+  if (threadIdx.x == 0) row_ptr[n] = carry;
+  for (int e = carry + threadIdx.x; e < n * K; e += blockDim.x) col[e] = -1;
+}
 
-  const int rows_per_step = 32 / K;  // K <= 32
-  const int sub = lane / K;
-  const bool lane_on = sub < rows_per_step;
-  const int slot = lane_on ? lane % K : lane;  // lanes past the last row never feed a row
-  const int rpw = (n + kTrWarps - 1) / kTrWarps;  // rows per warp
-  const int r_begin = min(n, warp * rpw), r_end = min(n, r_begin + rpw);
+__global__ void __launch_bounds__(kFillThreads)
+tr_fill_kernel(TransposeParams p) {
+  __shared__ int cur[kRangeKeys];
+  const TransposeLevel L = p.lv[level_of(p, blockIdx.x, kChunkGrid)];
+  const int local = blockIdx.x - L.cta_begin;
+  const int bh = local / L.nchunk, ch = local % L.nchunk;
+  const int n = L.n, K = p.K;
+  const int r0 = ch * L.rows, r1 = min(n, r0 + L.rows);
+  const int32_t* I = L.idx + (size_t)bh * n * K;
+  const int32_t* start = L.cnt + ((size_t)bh * L.nchunk + ch) * n;
+  const int32_t* row_ptr = L.row_ptr + (size_t)bh * (n + 1);
+  int32_t* col = L.col + (size_t)bh * n * K;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const RowLanes rl(K, lane);
 
-  // pass 1: counts (entries of kBatch steps are loaded before any is used,
-  // so their latencies overlap)
-  int flags = 0, my_below = 0;
-  for (int rb = r_begin; rb < r_end; rb += kBatch * rows_per_step) {
-    int cb[kBatch];
+  const int step = rl.rows_per_step * kBatch;
+  auto load_batch = [&](int rb, int (&cb)[kBatch]) {
 #pragma unroll
     for (int i = 0; i < kBatch; ++i) {
-      const int q = rb + i * rows_per_step + sub;
-      cb[i] = (lane_on && q < r_end) ? I[(size_t)q * K + slot] : -1;
+      const int q = rb + i * rl.rows_per_step + rl.sub;
+      cb[i] = (rl.on && q < r1) ? I[(size_t)q * K + rl.slot] : -1;
     }
+  };
+  for (int k0 = 0; k0 < n; k0 += kRangeKeys) {
+    const int len = min(n, k0 + kRangeKeys) - k0;
+    // cursors: the key's first slot plus this chunk's offset in its list,
+    // 8 pairs of loads in flight per thread
+    for (int e0 = threadIdx.x; e0 < len; e0 += 8 * kFillThreads) {
+      int t[8];
 #pragma unroll
-    for (int i = 0; i < kBatch; ++i) {
-      const int q = rb + i * rows_per_step + sub;
-      const bool on = lane_on && q < r_end;
-      const int c = cb[i];
-      const bool u = warp_row_used(c, slot, n, on, flags);
-      if (u && c >= c0 && c < c1) atomicAdd(&hist[warp][c - c0], 1);
-      if (u && c < c0) ++my_below;
-    }
-  }
-  my_below = __reduce_add_sync(0xffffffffu, my_below);
-  if (lane == 0) below[warp] = my_below;
-  __syncthreads();
-
-  // scan: offsets of the keys in [c0, c1)
-  if (threadIdx.x == 0) {
-    int b = 0;
-    for (int w = 0; w < kTrWarps; ++w) b += below[w];
-    below_total = b;
-  }
-  if (threadIdx.x < kTrRange) {
-    int tot = 0;
-    for (int w = 0; w < kTrWarps; ++w) tot += hist[w][threadIdx.x];
-    scan_buf[threadIdx.x] = tot;
-  }
-  __syncthreads();
-  // inclusive Hillis-Steele scan over 256 entries
-  for (int off = 1; off < kTrRange; off <<= 1) {
-    int v = 0;
-    if (threadIdx.x < kTrRange && threadIdx.x >= off) v = scan_buf[threadIdx.x - off];
-    __syncthreads();
-    if (threadIdx.x < kTrRange) scan_buf[threadIdx.x] += v;
-    __syncthreads();
-  }
-  if (threadIdx.x < kTrRange) {
-    const int t = threadIdx.x;
-    const int c = c0 + t;
-    const int excl = (t == 0) ? 0 : scan_buf[t - 1];
-    if (c < c1) {
-      const int start = below_total + excl;
-      row_ptr[c] = start;
-      int run = start;
-      for (int w = 0; w < kTrWarps; ++w) {
-        const int h = hist[w][t];
-        hist[w][t] = run;  // becomes warp w's cursor for key c
-        run += h;
+      for (int i = 0; i < 8; ++i) {
+        const int e = e0 + i * kFillThreads;
+        t[i] = (e < len) ? start[k0 + e] + row_ptr[k0 + e] : 0;
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = e0 + i * kFillThreads;
+        if (e < len) cur[e] = t[i];
       }
     }
-  }
-  const bool last_range = (c1 == n);
-  const int total = below_total + scan_buf[kTrRange - 1];
-  if (last_range && threadIdx.x == 0) row_ptr[n] = total;
-  __syncthreads();
-  if (last_range)
-    for (int e = total + threadIdx.x; e < n * K; e += blockDim.x) col[e] = -1;
-
-  // pass 2: fill
-  int dummy = 0;
-  for (int rb = r_begin; rb < r_end; rb += kBatch * rows_per_step) {
-    int cb[kBatch];
+    __syncthreads();
+    if (warp == 0) {
+      int dummy = 0;
+      int cb[kBatch], nb[kBatch];
+      load_batch(r0, cb);
+      for (int rb = r0; rb < r1; rb += step) {
+        load_batch(rb + step, nb);  // the next batch's loads overlap this batch
+        // the steps' screening and ranking are independent of one another
+        int key[kBatch], rank[kBatch];
+        unsigned peers[kBatch];
 #pragma unroll
-    for (int i = 0; i < kBatch; ++i) {
-      const int q = rb + i * rows_per_step + sub;
-      cb[i] = (lane_on && q < r_end) ? I[(size_t)q * K + slot] : -1;
-    }
+        for (int i = 0; i < kBatch; ++i) {
+          const int q = rb + i * rl.rows_per_step + rl.sub;
+          const int c = cb[i];
+          const bool u = warp_row_used(c, rl.slot, n, rl.on && q < r1, dummy, K);
+          key[i] = (u && c >= k0 && c < k0 + len) ? c - k0 : -1 - lane;  // -1 - lane matches nobody
+          peers[i] = __match_any_sync(0xffffffffu, key[i]);
+          rank[i] = __popc(peers[i] & ((1u << lane) - 1u));  // lower lanes hold lower rows
+        }
+        // the cursor updates run in step order
 #pragma unroll
-    for (int i = 0; i < kBatch; ++i) {
-      const int q = rb + i * rows_per_step + sub;
-      const bool on = lane_on && q < r_end;
-      const int c = cb[i];
-      const bool u = warp_row_used(c, slot, n, on, dummy);
-      const int key = (u && c >= c0 && c < c1) ? c : -2 - lane;  // -2 - lane matches nobody
-      const unsigned peers = __match_any_sync(0xffffffffu, key);
-      if (key >= 0) {
-        const unsigned lower = peers & ((1u << lane) - 1u);
-        col[hist[warp][key - c0] + __popc(lower)] = q;
+        for (int i = 0; i < kBatch; ++i) {
+          const int q = rb + i * rl.rows_per_step + rl.sub;
+          if (key[i] >= 0) col[cur[key[i]] + rank[i]] = q;
+          __syncwarp();
+          if (key[i] >= 0 && lane == 31 - __clz(peers[i])) cur[key[i]] += __popc(peers[i]);
+          __syncwarp();
+        }
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) cb[i] = nb[i];
       }
-      __syncwarp();
-      if (key >= 0 && lane == 31 - __clz(peers)) hist[warp][key - c0] += __popc(peers);
-      __syncwarp();
     }
-  }
-  if (local % L.ranges == 0) {
-    flags = __reduce_or_sync(0xffffffffu, flags);
-    if (lane == 0) report_status(p.status, flags);
+    __syncthreads();  // cur is restaged for the next key range
   }
 }
 
 }  // namespace
 
+// Rows per chunk for a level of n query rows: at most kMaxChunks chunks, at
+// least 64 rows each (the workspace holds nchunk * n counts per (b, h)).
+void transpose_chunking(int n, int* nchunk, int* rows) {
+  int c = (n + 63) / 64;
+  if (c > kMaxChunks) c = kMaxChunks;
+  if (c < 1) c = 1;
+  *rows = (n + c - 1) / c;
+  *nchunk = (n + *rows - 1) / *rows;
+}
+
 cudaError_t launch_transpose(const TransposeParams& p, cudaStream_t s) {
-  const int total = p.lv[p.nlev - 1].cta_begin + p.BH * p.lv[p.nlev - 1].ranges;
-  transpose_kernel<<<total, kTrWarps * 32, 0, s>>>(p);
+  const TransposeLevel& last = p.lv[p.nlev - 1];
+  const int chunks = last.cta_begin + p.BH * last.nchunk;
+  const int tiles = last.tile_begin + p.BH * ((last.n + kPrefixKeys - 1) / kPrefixKeys);
+  const int scans = last.scan_begin + p.BH;
+  tr_count_kernel<<<chunks, kCountThreads, 0, s>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  tr_prefix_kernel<<<tiles, kPrefixThreads, 0, s>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  tr_scan_kernel<<<scans, kScanThreads, 0, s>>>(p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  tr_fill_kernel<<<chunks, kFillThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
+
+int transpose_prefix_tiles(int n) { return (n + kPrefixKeys - 1) / kPrefixKeys; }
 
 }  // namespace llsa

@@ -58,7 +58,7 @@ enum {
   LLSA_ERR_INVALID_ARG = 1, /* NULL pointer, bad shape, N not a multiple of 16^L, ... */
   LLSA_ERR_UNSUPPORTED = 2, /* D not in {64, 128}, topk > 32, L > 6, ... */
   LLSA_ERR_LAUNCH = 3,      /* a kernel launch failed (cudaGetLastError) */
-  LLSA_ERR_WORKSPACE = 4    /* workspace smaller than llsa_bwd_workspace_bytes() */
+  LLSA_ERR_WORKSPACE = 4    /* workspace smaller than the matching *_workspace_bytes() */
 };
 
 /* descriptor flags */
@@ -159,16 +159,29 @@ LLSA_API int llsa_attn_fwd(const llsa_desc* desc, const void* q, const void* k, 
                   int32_t* dev_status, void* stream);
 
 /*
+ * llsa_transpose_workspace_bytes - device scratch size that
+ * llsa_index_transpose needs for desc (0 on an invalid desc): per level,
+ * B*H*nchunk*N_l int32 counts with nchunk <= 32 row chunks.
+ */
+LLSA_API size_t llsa_transpose_workspace_bytes(const llsa_desc* desc);
+
+/*
  * llsa_index_transpose - sparse index transpose (Step 4; Building Blocks:
  * Sparse Index Transpose).
  *   For each level l = 1..L and (b, h): count the query tokens that kept each
  *   key token, prefix-sum the counts into row_ptr, and list the query tokens
  *   of each key in ascending order in col.  No dense mask is formed; the
  *   result is deterministic and uses no global atomics.
- *   idx: I(1..L).  out: CSR of every level, written.  dev_status: may be NULL.
+ *   idx: I(1..L), entries screened as the conventions above state.
+ *   out: CSR of every level, written: row_ptr[l] int32 [B, H, N_l + 1],
+ *   col[l] int32 [B, H, N_l * K] (slots past row_ptr[N_l] set to -1).
+ *   ws: device scratch of at least llsa_transpose_workspace_bytes(desc)
+ *   bytes, 256-byte aligned, not read before it is written (a smaller or
+ *   missing one gives LLSA_ERR_WORKSPACE / LLSA_ERR_INVALID_ARG before any
+ *   launch).  dev_status: may be NULL.
  */
 LLSA_API int llsa_index_transpose(const llsa_desc* desc, const llsa_indices* idx, const llsa_csr* out,
-                         int32_t* dev_status, void* stream);
+                         void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
 
 /*
  * llsa_bwd_workspace_bytes - device scratch size that llsa_attn_bwd needs

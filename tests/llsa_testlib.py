@@ -85,7 +85,7 @@ def run_gpu(B, H, N, D, L, topk, dtype, inputs, level_w=None, ext_idx=None, bwd=
     llsa.llsa_attn_fwd(desc, t["q"].data_ptr(), t["k"].data_ptr(), t["v"].data_ptr(), bufs.pyramid,
                        bufs.indices, o.data_ptr(), lse.data_ptr(), st, stream)
     if bwd:
-        llsa.llsa_index_transpose(desc, bufs.indices, bufs.csr, st, stream)
+        llsa.llsa_index_transpose(desc, bufs.indices, bufs.csr, bufs.tr_ws.data_ptr(), bufs.tr_ws_bytes, st, stream)
         dq, dk, dv = torch.empty_like(o), torch.empty_like(o), torch.empty_like(o)
         llsa.llsa_attn_bwd(desc, t["q"].data_ptr(), t["k"].data_ptr(), t["v"].data_ptr(), bufs.pyramid,
                            o.data_ptr(), lse.data_ptr(), t["do"].data_ptr(), bufs.indices, bufs.csr,

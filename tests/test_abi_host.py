@@ -65,7 +65,8 @@ def test_bad_descriptors_are_rejected_before_launch(lib, kw, status):
     fake = 256  # never dereferenced: the check fails first
     assert llsa.llsa_pool(d, fake, fake, fake, pyr, check=False) == status
     assert llsa.llsa_select(d, pyr, ind, check=False) == status
-    assert llsa.llsa_index_transpose(d, ind, csr, check=False) == status
+    assert llsa.llsa_index_transpose(d, ind, csr, 256, 1 << 40, check=False) == status
+    assert llsa.llsa_transpose_workspace_bytes(d) == 0
     assert llsa.llsa_bwd_workspace_bytes(d) == 0
 
 
@@ -76,7 +77,7 @@ def test_null_buffers_are_rejected(lib):
     assert llsa.llsa_pool(d, 256, 256, 256, pyr, check=False) == llsa.ERR_INVALID_ARG
     assert llsa.llsa_select(d, pyr, ind, check=False) == llsa.ERR_INVALID_ARG
     assert llsa.llsa_attn_fwd(d, 256, 256, 256, pyr, ind, 256, 256, check=False) == llsa.ERR_INVALID_ARG
-    assert llsa.llsa_index_transpose(d, ind, csr, check=False) == llsa.ERR_INVALID_ARG
+    assert llsa.llsa_index_transpose(d, ind, csr, 256, 1 << 40, check=False) == llsa.ERR_INVALID_ARG
     with pytest.raises(llsa.LlsaError):
         llsa.llsa_select(d, pyr, ind)
 
@@ -88,6 +89,7 @@ def test_workspace_size_and_checks(lib):
     want = r256(B * H * N * 4)
     want += sum(r256(B * H * (N // 128) * K * 2 * D * 4) for _ in range(2, L + 1))
     want += sum(r256(B * H * (N // 16**l) * 2 * D * 4) for l in range(2, L + 1))
+    want += 256  # the key-major pass's work counter
     assert llsa.llsa_bwd_workspace_bytes(d) == want
     # fill every pointer with a fake non-null value: the size check fails first
     pyr, ind, csr = llsa.LlsaPyramid(), llsa.LlsaIndices(), llsa.LlsaCsr()
@@ -99,6 +101,33 @@ def test_workspace_size_and_checks(lib):
     st = llsa.llsa_attn_bwd(d, 256, 256, 256, pyr, 256, 256, 256, ind, csr, 256, 256, 256,
                             260, want, check=False)
     assert st == llsa.ERR_INVALID_ARG  # workspace not 256-byte aligned
+
+
+def _transpose_ws_bytes(B, H, N, L):
+    # per level: nchunk row chunks (at most 32, at least 64 rows each), one
+    # int32 count per (b, h, chunk, key), each level 256-byte aligned
+    total = 0
+    for l in range(1, L + 1):
+        n = N // 16**l
+        c = min(32, max(1, (n + 63) // 64))
+        rows = (n + c - 1) // c
+        c = (n + rows - 1) // rows
+        total += (B * H * c * n * 4 + 255) // 256 * 256
+    return total
+
+
+@pytest.mark.parametrize("shape", [(1, 2, 4096, 3), (2, 3, 1024, 2), (1, 1, 65536, 4), (1, 2, 256, 2)])
+def test_transpose_workspace_size_and_checks(lib, shape):
+    B, H, N, L = shape
+    d = _desc(B=B, H=H, N=N, L=L)
+    want = _transpose_ws_bytes(B, H, N, L)
+    assert llsa.llsa_transpose_workspace_bytes(d) == want
+    ind, csr = llsa.LlsaIndices(), llsa.LlsaCsr()
+    for l in range(1, L + 1):
+        ind.idx[l] = csr.row_ptr[l] = csr.col[l] = 256
+    assert llsa.llsa_index_transpose(d, ind, csr, 256, want - 1, check=False) == llsa.ERR_WORKSPACE
+    assert llsa.llsa_index_transpose(d, ind, csr, 260, want, check=False) == llsa.ERR_INVALID_ARG
+    assert llsa.llsa_index_transpose(d, ind, csr, None, want, check=False) == llsa.ERR_INVALID_ARG
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):

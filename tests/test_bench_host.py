@@ -1,0 +1,92 @@
+"""Host-side logic of bench.py: the algorithmic work behind the roofline
+fractions, the launch count, the committed-traffic lookup and the
+max-over-ranks timing of multi-process runs (gloo, two ranks, CPU)."""
+
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+from hierarchical_top_sparse_llsa_b200 import workloads
+
+
+def test_algorithmic_work_headline():
+    # 256x256 pixels: B=1, H=16, N=65536, D=64, L=3, K=8 (144 keys per query)
+    w = workloads.WORKLOADS["img256_bf16"]
+    assert w.keys_per_query() == 144
+    work = bench.algorithmic_work(w)
+    pairs = 16 * 65536 * 144
+    assert work["fwd"]["flops"] == 4 * 64 * pairs and abs(work["fwd"]["flops"] - 3.87e10) < 0.01e10
+    assert work["bwd"]["flops"] == 10 * 64 * pairs
+    fine = 16 * 65536 * 64 * 2
+    assert work["fwd"]["bytes"] == 4 * fine + 16 * 65536 * 4
+    assert abs(work["pool"]["bytes"] - 440e6) < 10e6
+    assert abs(work["transpose"]["bytes"] - 4.8e6) < 0.2e6
+
+
+def test_launch_count_per_step():
+    assert bench.launches_per_step(3) == {"pool": 2, "select": 3, "fwd": 1, "transpose": 4, "bwd": 5}
+    assert sum(bench.launches_per_step(2).values()) == 1 + 2 + 1 + 4 + 3
+
+
+def _fake_tree(root, src):
+    os.makedirs(os.path.join(root, "hierarchical_top_sparse_llsa_b200", "csrc"))
+    os.makedirs(os.path.join(root, "include"))
+    os.makedirs(os.path.join(root, "profiles"))
+    with open(os.path.join(root, "hierarchical_top_sparse_llsa_b200", "csrc", "k.cu"), "w") as f:
+        f.write(src)
+    with open(os.path.join(root, "include", "llsa.h"), "w") as f:
+        f.write("/* header */\n")
+
+
+def test_committed_traffic_is_dropped_when_sources_change(tmp_path, monkeypatch):
+    root = str(tmp_path)
+    _fake_tree(root, "__global__ void k() {}\n")
+    monkeypatch.setattr(bench, "ROOT", root)
+    digest = bench.sources_digest()
+    with open(os.path.join(root, "profiles", "dram_traffic_wl.md"), "w") as f:
+        f.write("# summary\n\n```json\n"
+                '{"sources_sha1": "%s", "stages": {"bwd": {"dram_bytes_per_call": 12345}}}\n'
+                "```\n" % digest)
+    assert bench.committed_traffic("wl", "bwd") == 12345
+    assert bench.committed_traffic("wl", "fwd") is None
+    assert bench.committed_traffic("other", "bwd") is None
+    with open(os.path.join(root, "hierarchical_top_sparse_llsa_b200", "csrc", "k.cu"), "a") as f:
+        f.write("// changed\n")
+    assert bench.committed_traffic("wl", "bwd") is None
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    import torch
+    import torch.distributed as dist
+
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank, world_size=world)
+    try:
+        # rank r is slow on the first timing and fast on the second
+        got = bench.max_over_ranks(torch, dist, [1.0 + rank, 10.0 - rank], "cpu")
+        out[rank] = got
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.timeout(120)
+def test_max_over_ranks_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    with ctx.Manager() as mgr:
+        out = mgr.dict()
+        port = _free_port()
+        procs = [ctx.Process(target=_rank_main, args=(r, 2, port, out)) for r in range(2)]
+        for p in procs:
+            p.start()
+        for p in procs:
+            p.join(100)
+        assert all(p.exitcode == 0 for p in procs)
+        assert out[0] == [2.0, 10.0] and out[1] == [2.0, 10.0]

@@ -37,7 +37,8 @@ def _problem(name):
     lse = torch.empty(w.B, w.H, w.N, dtype=torch.float32, device="cuda")
     llsa.llsa_attn_fwd(desc, q, k, v, bufs.pyramid, bufs.indices, o.data_ptr(), lse.data_ptr(),
                        bufs.status.data_ptr(), s)
-    llsa.llsa_index_transpose(desc, bufs.indices, bufs.csr, bufs.status.data_ptr(), s)
+    llsa.llsa_index_transpose(desc, bufs.indices, bufs.csr, bufs.tr_ws.data_ptr(), bufs.tr_ws_bytes,
+                              bufs.status.data_ptr(), s)
     return w, t, desc, bufs, o, lse, s
 
 
