@@ -223,21 +223,25 @@ __global__ void bwd_coarse_reduce_kernel(AttnParams p, int l) {
       s_slot[e] = slot;
     }
     __syncthreads();
-    for (int e = 0; e < cnt; ++e) {
-      const int slot = s_slot[e];
-      if (slot < 0) continue;
-      const float* src = part + ((size_t)s_q[e] * span * K + slot) * 2 * D;
-      const size_t stride = (size_t)K * 2 * D;  // next group, same slot
-      int a = 0;
-      for (; a + 4 <= nsum; a += 4) {
-        const float x0 = src[(a + 0) * stride], x1 = src[(a + 1) * stride];
-        const float x2 = src[(a + 2) * stride], x3 = src[(a + 3) * stride];
-        acc += x0;
-        acc += x1;
-        acc += x2;
-        acc += x3;
+    // entries in batches of 8 whose loads are all in flight before the sums,
+    // which still run in entry order, then group order (nsum is 2 at level 2
+    // and 1 above)
+    const size_t stride = (size_t)K * 2 * D;  // next group, same slot
+    for (int eb = 0; eb < cnt; eb += 8) {
+      float x0[8], x1[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int e = eb + i;
+        const int slot = (e < cnt) ? s_slot[e] : -1;
+        const float* src = part + ((size_t)(slot >= 0 ? s_q[e] : 0) * span * K + (slot >= 0 ? slot : 0)) * 2 * D;
+        x0[i] = (slot >= 0) ? src[0] : 0.f;
+        x1[i] = (slot >= 0 && nsum > 1) ? src[stride] : 0.f;
       }
-      for (; a < nsum; ++a) acc += src[a * stride];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        acc += x0[i];
+        acc += x1[i];
+      }
     }
   }
   p.coarse[l][((size_t)bh * nl + c) * 2 * D + t] = acc;

@@ -11,8 +11,10 @@
 // is read from shared memory 4 times rather than 16.
 //
 // Score: fp32, d = 0..D-1 left to right, one rounding per multiply and per
-// add (explicit __fmul_rn/__fadd_rn: no contraction into FMA), so scores are
-// reproducible bit for bit and the selected indices are exact.
+// add (no contraction into FMA), so scores are reproducible bit for bit and
+// the selected indices are exact.  The products and sums run as packed pairs
+// (sm_100 mul/add .f32x2: each half rounded exactly as the scalar .rn op),
+// two candidates per instruction.
 // Top-K: each (score, index) pair is packed into one 64-bit key that orders
 // by score (with -0 == +0) and then by lower index; K rounds of a warp-wide
 // maximum (two redux.sync on 32-bit halves) pick the winners, merging the
@@ -29,6 +31,28 @@ constexpr int kSelWarps = 4;
 constexpr int kSelThreads = kSelWarps * 32;
 constexpr int kSelChunk = 128;   // candidates scored per pass
 constexpr int kSelItems = kSelChunk / 32;
+
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t d;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(d) : "r"(__float_as_uint(lo)), "r"(__float_as_uint(hi)));
+  return d;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t x, float& lo, float& hi) {
+  uint32_t a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(a), "=r"(b) : "l"(x));
+  lo = __uint_as_float(a);
+  hi = __uint_as_float(b);
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
 
 __device__ __forceinline__ uint64_t pack_key(float s, int idx) {
   s = __fadd_rn(s, 0.0f);  // -0 -> +0, so that equal scores compare equal
@@ -81,7 +105,7 @@ select_kernel(SelectParams p) {
   // the 16 query rows, transposed
   const float* qbase = p.ql + ((size_t)bh * n + (size_t)grp * kSelQ) * D;
   for (int e = tid; e < kSelQ * (D / 4); e += kSelThreads) {
-    const int r = e / (D / 4), c4 = e % (D / 4);
+    const int r = e % kSelQ, c4 = e / kSelQ;  // lanes walk the rows: conflict-free stores
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (grp * kSelQ + r < n) v = *reinterpret_cast<const float4*>(qbase + (size_t)r * D + c4 * 4);
     qsT[(4 * c4 + 0) * QLD + r] = v.x;
@@ -102,69 +126,96 @@ select_kernel(SelectParams p) {
   for (int c0 = 0; c0 < C; c0 += kSelChunk) {
     const int cn = min(kSelChunk, C - c0);
     __syncthreads();
-    for (int e = tid; e < kSelChunk * (D / 4); e += kSelThreads) {
+    // all of this thread's row loads are issued before any is stored, so
+    // their latencies overlap
+    constexpr int kStageIters = kSelChunk * (D / 4) / kSelThreads;
+    float4 kv4[kStageIters];
+#pragma unroll
+    for (int it = 0; it < kStageIters; ++it) {
+      const int e = tid + it * kSelThreads;
       const int r = e % kSelChunk, c4 = e / kSelChunk;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      kv4[it] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (r < cn) {
         const int j = c0 + r;
         const int c = top ? j : parents[j / kBlock] * kBlock + (j % kBlock);
-        v = *reinterpret_cast<const float4*>(kbase + (size_t)c * D + c4 * 4);
+        kv4[it] = *reinterpret_cast<const float4*>(kbase + (size_t)c * D + c4 * 4);
         if (c4 == 0) cid[r] = c;
       }
-      ksT[(4 * c4 + 0) * CLD + r] = v.x;
-      ksT[(4 * c4 + 1) * CLD + r] = v.y;
-      ksT[(4 * c4 + 2) * CLD + r] = v.z;
-      ksT[(4 * c4 + 3) * CLD + r] = v.w;
+    }
+#pragma unroll
+    for (int it = 0; it < kStageIters; ++it) {
+      const int e = tid + it * kSelThreads;
+      const int r = e % kSelChunk, c4 = e / kSelChunk;
+      ksT[(4 * c4 + 0) * CLD + r] = kv4[it].x;
+      ksT[(4 * c4 + 1) * CLD + r] = kv4[it].y;
+      ksT[(4 * c4 + 2) * CLD + r] = kv4[it].z;
+      ksT[(4 * c4 + 3) * CLD + r] = kv4[it].w;
     }
     __syncthreads();
-    // scores: d = 0..D-1 in order, one rounding per multiply and per add
-    float acc[4][4];
+    // scores: d = 0..D-1 in order, one rounding per multiply and per add;
+    // acc[a][h] holds candidates 4cg + 2h, 4cg + 2h + 1 of query 4qg + a
+    uint64_t acc[4][2];
 #pragma unroll
     for (int d = 0; d < D; ++d) {
       const float4 qv = *reinterpret_cast<const float4*>(qsT + d * QLD + 4 * qg);
       const float4 kv = *reinterpret_cast<const float4*>(ksT + d * CLD + 4 * cg);
+      const uint64_t k01 = f2_pack(kv.x, kv.y), k23 = f2_pack(kv.z, kv.w);
       const float qq[4] = {qv.x, qv.y, qv.z, qv.w};
-      const float kk[4] = {kv.x, kv.y, kv.z, kv.w};
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          acc[a][c] = (d == 0) ? __fmul_rn(qq[a], kk[c]) : __fadd_rn(acc[a][c], __fmul_rn(qq[a], kk[c]));
+      for (int a = 0; a < 4; ++a) {
+        const uint64_t q2 = f2_pack(qq[a], qq[a]);
+        const uint64_t m01 = f2_mul(q2, k01), m23 = f2_mul(q2, k23);
+        acc[a][0] = (d == 0) ? m01 : f2_add(acc[a][0], m01);
+        acc[a][1] = (d == 0) ? m23 : f2_add(acc[a][1], m23);
+      }
     }
 #pragma unroll
-    for (int a = 0; a < 4; ++a)
-      *reinterpret_cast<float4*>(sc + (4 * qg + a) * kSelChunk + 4 * cg) =
-          make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+    for (int a = 0; a < 4; ++a) {
+      float4 o;
+      f2_unpack(acc[a][0], o.x, o.y);
+      f2_unpack(acc[a][1], o.z, o.w);
+      *reinterpret_cast<float4*>(sc + (4 * qg + a) * kSelChunk + 4 * cg) = o;
+    }
     __syncthreads();
-    // Top-K merge, one query of this warp at a time
+    // Top-K merge: the warp's queries advance together, so their K rounds of
+    // warp-wide maxima are independent chains
+    constexpr int QW = kSelQ / kSelWarps;
+    uint64_t item[QW][kSelItems + 1];
 #pragma unroll
-    for (int qi = 0; qi < kSelQ / kSelWarps; ++qi) {
-      const int ql = warp * (kSelQ / kSelWarps) + qi;
-      uint64_t item[kSelItems + 1];
+    for (int qi = 0; qi < QW; ++qi) {
+      const int ql = warp * QW + qi;
 #pragma unroll
       for (int it = 0; it < kSelItems; ++it) {
         const int j = lane + 32 * it;
-        item[it] = (j < cn) ? pack_key(sc[ql * kSelChunk + j], cid[j]) : 0;
+        item[qi][it] = (j < cn) ? pack_key(sc[ql * kSelChunk + j], cid[j]) : 0;
       }
-      item[kSelItems] = (lane < K) ? run[qi] : 0;
-      uint64_t next = 0;
-      for (int r = 0; r < K; ++r) {
+      item[qi][kSelItems] = (lane < K) ? run[qi] : 0;
+    }
+    uint64_t next[QW];
+#pragma unroll
+    for (int qi = 0; qi < QW; ++qi) next[qi] = 0;
+    for (int r = 0; r < K; ++r) {
+#pragma unroll
+      for (int qi = 0; qi < QW; ++qi) {
         uint64_t mine = 0;
         int arg = 0;
 #pragma unroll
         for (int it = 0; it <= kSelItems; ++it)
-          if (item[it] > mine) { mine = item[it]; arg = it; }
-        const uint64_t best = warp_max_u64(mine);
-        if (best == 0) break;  // uniform: no candidates left
-        if (mine == best) {
+          if (item[qi][it] > mine) {
+            mine = item[qi][it];
+            arg = it;
+          }
+        const uint64_t best = warp_max_u64(mine);  // 0: no candidates left
+        if (best != 0 && mine == best) {
 #pragma unroll
           for (int it = 0; it <= kSelItems; ++it)
-            if (it == arg) item[it] = 0;
+            if (it == arg) item[qi][it] = 0;
         }
-        if (lane == r) next = best;
+        if (lane == r) next[qi] = best;
       }
-      run[qi] = next;
     }
+#pragma unroll
+    for (int qi = 0; qi < QW; ++qi) run[qi] = next[qi];
   }
   // ascending index order; the kept entries are lanes 0..cnt-1
 #pragma unroll
