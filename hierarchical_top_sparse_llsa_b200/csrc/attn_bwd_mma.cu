@@ -16,14 +16,18 @@
 // small dK entries 3x (dV 1.5x) outside a 2e-2 relative band.  dQ, a sum
 // over keys, keeps a single bf16 dS (worst case 0.45 of that band).
 // Coarse keys then give dQ their share and, per CTA, the partials
-// sum_i dS_ij q_i and sum_i P_ij dO_i: each warp forms its block's part with
-// MMAs on register transposes (movmatrix), and the CTA adds the 8 parts in a
-// fixed warp order, so no atomics are used.
+// sum_i dS_ij q_i and sum_i P_ij dO_i over the 8 blocks' queries: the warps
+// exchange P and dS (bf16 hi + lo) through shared memory and each warp sums
+// the 8 blocks for its own output columns with MMAs in warp order, so no
+// atomics are used.
 //
-// Pass 3, key-major (bwd_kv_mma_kernel): one warp per 16-token key block walks
-// its row of the level-1 key-major lists (query blocks, ascending).  With the
-// key block as the MMA's M: S^T = K Q^T, dP^T = V dO^T, dV += P^T dO,
-// dK += dS^T Q.  The epilogue adds every coarse gradient divided by 16^l.
+// Pass 3, key-major (bwd_kv_mma_kernel): persistent single-warp CTAs take
+// 16-token key blocks from a work counter and walk each block's row of the
+// level-1 key-major lists (query blocks, ascending).  With the key block as
+// the MMA's M: S^T = K Q^T, dP^T = V dO^T, dV += P^T dO, dK += dS^T Q.  The
+// next row's K/V, coarse gradient rows and first Q/dO tiles are loaded
+// before the current row's epilogue, which adds every coarse gradient
+// divided by 16^l.
 // (Pass 2, the per-level coarse reduce, is shared with the fp32 path.)
 
 #include <math.h>
@@ -38,21 +42,44 @@ namespace llsa {
 namespace {
 
 constexpr int kQWarps = 8;   // query blocks per CTA in pass 1 (one partial group)
-constexpr int kRing = 2;
+constexpr int kRing = 2;    // K/V ring stages per warp in pass 1
+#ifndef LLSA_KV_RING
+#define LLSA_KV_RING 2
+#endif
+constexpr int kRingKV = LLSA_KV_RING;  // Q/dO ring stages in pass 3
 constexpr float kLog2e = 1.4426950408889634f;
 
 // P = exp2(S * sc2 + lw - lse2) on a 16x16 tile (rows g, g+8 of the query
-// side); rows with lse = -inf get P = 0.
+// side); rows with lse = -inf get P = 0.  Pairs of columns run as packed
+// f32x2 operations (bit-identical to the scalar fma).
 __device__ __forceinline__ void probs_rows(const float (&s)[2][4], const float (&lw)[2][2], float sc2,
                                            float lse_g, float lse_g8, float (&P)[2][4]) {
+  const float n0 = (lse_g == -INFINITY) ? -INFINITY : -lse_g;
+  const float n1 = (lse_g8 == -INFINITY) ? -INFINITY : -lse_g8;
+  const uint64_t sc = f2_make(sc2, sc2);
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt) {
+    const float2 a = f2_split(f2_fma(f2_make(s[nt][0], s[nt][1]), sc, f2_make(lw[nt][0] + n0, lw[nt][1] + n0)));
+    const float2 b = f2_split(f2_fma(f2_make(s[nt][2], s[nt][3]), sc, f2_make(lw[nt][0] + n1, lw[nt][1] + n1)));
+    P[nt][0] = ex2_approx(a.x);
+    P[nt][1] = ex2_approx(a.y);
+    P[nt][2] = ex2_approx(b.x);
+    P[nt][3] = ex2_approx(b.y);
+  }
+}
+
+// dS = P (dP - Delta) in place of P, rows g (delta_g) and g+8 (delta_g8)
+__device__ __forceinline__ void ds_rows(float (&P)[2][4], const float (&dp)[2][4], float delta_g,
+                                        float delta_g8) {
+  const uint64_t d0 = f2_make(delta_g, delta_g), d1 = f2_make(delta_g8, delta_g8);
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float lse = (e < 2) ? lse_g : lse_g8;
-      const float x = fmaf(s[nt][e], sc2, lw[nt][e & 1] - lse);
-      P[nt][e] = (lse == -INFINITY) ? 0.f : ex2_approx(x);
-    }
+  for (int nt = 0; nt < 2; ++nt) {
+    const float2 a = f2_split(f2_mul(f2_make(P[nt][0], P[nt][1]), f2_sub(f2_make(dp[nt][0], dp[nt][1]), d0)));
+    const float2 b = f2_split(f2_mul(f2_make(P[nt][2], P[nt][3]), f2_sub(f2_make(dp[nt][2], dp[nt][3]), d1)));
+    P[nt][0] = a.x;
+    P[nt][1] = a.y;
+    P[nt][2] = b.x;
+    P[nt][3] = b.y;
   }
 }
 
@@ -61,27 +88,6 @@ __device__ __forceinline__ void pack_frag(const float (&x)[2][4], uint32_t (&a)[
   a[1] = pack_bf16(x[0][2], x[0][3]);
   a[2] = pack_bf16(x[1][0], x[1][1]);
   a[3] = pack_bf16(x[1][2], x[1][3]);
-}
-
-// A fragment of the transpose of the 16x16 matrix whose A fragment is `a`.
-__device__ __forceinline__ void transpose_frag(const uint32_t (&a)[4], uint32_t (&t)[4]) {
-  t[0] = movmatrix_t(a[0]);
-  t[1] = movmatrix_t(a[2]);
-  t[2] = movmatrix_t(a[1]);
-  t[3] = movmatrix_t(a[3]);
-}
-
-// acc (16 x D) = A (16 x 16) . X (16 x D) where X's A fragments are `xa`
-// (X rows = the contraction index): the B fragments of X are the transposes
-// of its 8x8 sub-blocks.
-template <int D>
-__device__ __forceinline__ void mm_with_rowfrags(const uint32_t (&a)[4], const uint32_t (&xa)[D / 16][4],
-                                                 float (&acc)[D / 8][4]) {
-#pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    mma_bf16(acc[2 * kk], a, movmatrix_t(xa[kk][0]), movmatrix_t(xa[kk][1]));
-    mma_bf16(acc[2 * kk + 1], a, movmatrix_t(xa[kk][2]), movmatrix_t(xa[kk][3]));
-  }
 }
 
 template <int D>
@@ -274,10 +280,7 @@ bwd_q_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
           delta_g8 = dp1;
         }
       } else {  // sweep 2: dQ += dS K
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-          for (int e = 0; e < 4; ++e) P[nt][e] *= d_cur[nt][e] - ((e < 2) ? delta_g : delta_g8);
+        ds_rows(P, d_cur, delta_g, delta_g8);
         uint32_t dsa[4];
         pack_frag(P, dsa);
         pv_tile<D>(dsa, ring_k(st), lane, dq);
@@ -330,10 +333,20 @@ bwd_q_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
     }
   }
 
-  // coarse keys: dQ share and the per-CTA partials, reduced in warp order
+  // Coarse keys: this block's dQ share, then the CTA's partials
+  //   part_dk[key] = scale * sum_i dS_i,key q_i,  part_dv[key] = sum_i P_i,key dO_i
+  // over the 8 blocks' 128 queries.  Each warp leaves P and dS (bf16 hi + lo,
+  // rows = its queries, columns = the 16 coarse keys) in shared memory; after
+  // one barrier, warp w' owns D/32 output n-tiles of one of the two partials
+  // and sums the 8 blocks in warp order with MMAs (the 16 queries of a block
+  // are the contraction), so no fp32 staging or cross-warp add is needed.
+  constexpr int XROW = 48;          // bytes per row of a 16 x 16 bf16 exchange matrix (conflict-free)
+  constexpr int XMAT = 16 * XROW;   // one matrix
+  constexpr int NTW = D / 32;       // output n-tiles per warp
   const int NG = n1 / kQWarps;
-  float* stage = reinterpret_cast<float*>(wbase + 2 * TILE);  // [2][16][D] fp32, reuses this warp's ring
+  auto xbuf = [&](int w) { return smem_u32(sm + (size_t)w * TILE * (2 + 2 * kRing) + 2 * TILE); };
   for (int ct = 0; ct < ncpad; ++ct) {
+    uint32_t xw = xbuf(warp);  // [dS hi | dS lo | P hi | P lo], reuses this warp's ring
     if (active && ok) {
       float s[2][4], dpv[2][4], P[2][4], dS[2][4], lw[2][2];
 #pragma unroll
@@ -348,59 +361,66 @@ bwd_q_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int e = 0; e < 4; ++e) dS[nt][e] = P[nt][e] * (dpv[nt][e] - ((e < 2) ? delta_g : delta_g8));
-      uint32_t qa[D / 16][4], da[D / 16][4];
-      load_a_frags<D>(qt, lane, qa);
-      load_a_frags<D>(dot, lane, da);
-      uint32_t dsh[4], dsl[4], ph[4], pl[4], dsth[4], dstl[4], pth[4], ptl[4];
-      split_frag(dS, dsh, dsl);
-      split_frag(P, ph, pl);
-      pv_tile2<D>(dsh, dsl, smem_u32(ck) + ct * TILE, lane, dq);
-      transpose_frag(dsh, dsth);
-      transpose_frag(dsl, dstl);
-      transpose_frag(ph, pth);
-      transpose_frag(pl, ptl);
-      // part (16 coarse keys x D): rows g, g+8 of the transposed products
-      {
-        float acc[NT][4];
+      uint32_t frag[4][4];  // dS hi, dS lo, P hi, P lo (A-fragment order)
+      split_frag(dS, frag[0], frag[1]);
+      split_frag(P, frag[2], frag[3]);
+      pv_tile2<D>(frag[0], frag[1], smem_u32(ck) + ct * TILE, lane, dq);
+      // fragment register i holds rows g (i even) / g+8 (i odd), columns 8(i>>1) + 2t, +1
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-        mm_with_rowfrags<D>(dsth, qa, acc);
-        mm_with_rowfrags<D>(dstl, qa, acc);
+      for (int m = 0; m < 4; ++m)
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          *reinterpret_cast<float2*>(stage + g * D + 8 * nt + 2 * t) = make_float2(acc[nt][0], acc[nt][1]);
-          *reinterpret_cast<float2*>(stage + (g + 8) * D + 8 * nt + 2 * t) = make_float2(acc[nt][2], acc[nt][3]);
+        for (int i = 0; i < 4; ++i) {
+          const int row = g + 8 * (i & 1), col = 8 * (i >> 1) + 2 * t;
+          asm volatile("st.shared.u32 [%0], %1;" ::"r"(xw + m * XMAT + row * XROW + col * 2), "r"(frag[m][i])
+                       : "memory");
         }
-      }
-      {
-        float acc[NT][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
-        mm_with_rowfrags<D>(pth, da, acc);
-        mm_with_rowfrags<D>(ptl, da, acc);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          *reinterpret_cast<float2*>(stage + 16 * D + g * D + 8 * nt + 2 * t) = make_float2(acc[nt][0], acc[nt][1]);
-          *reinterpret_cast<float2*>(stage + 16 * D + (g + 8) * D + 8 * nt + 2 * t) = make_float2(acc[nt][2], acc[nt][3]);
-        }
-      }
     } else {
-      float* stg = stage;
-      for (int e = lane; e < 32 * D; e += 32) stg[e] = 0.f;
+      for (int e = lane; e < 4 * XMAT / 4; e += 32)
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(xw + 4 * e), "r"(0u) : "memory");
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < 32 * D; e += blockDim.x) {
-      const int kv = e / (16 * D), key = (e / D) % 16, d = e % D;
-      const int ck_idx = ct * 16 + key;
-      if (ck_idx >= nc) continue;
-      float a = 0.f;
-      for (int w = 0; w < kQWarps; ++w)
-        a += reinterpret_cast<const float*>(sm + (size_t)w * TILE * (2 + 2 * kRing) + 2 * TILE)[e];
-      const int l = clist[ck_idx] >> 24;
-      float* part = p.part[l] + ((((size_t)bh * NG + grp) * K + cslot[ck_idx]) * 2 + kv) * D + d;
-      *part = (kv == 0) ? a * p.scale : a;
+    {
+      const int kv = warp >> 2;           // 0: dK partial (dS, Q), 1: dV partial (P, dO)
+      const int j0 = NTW * (warp & 3);    // first output n-tile
+      float acc[NTW][4];
+#pragma unroll
+      for (int j = 0; j < NTW; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+      const int mi = lane >> 3;
+      // A = X^T (keys x queries) from X (queries x keys, row-major): transposed loads
+      const int xr = (mi >> 1) * 8 + (lane & 7), xc = (mi & 1) * 8;
+      const int vrow = (mi & 1) * 8 + (lane & 7), vc = mi >> 1;
+      for (int w = 0; w < kQWarps; ++w) {
+        const uint32_t xs = xbuf(w) + (2 * kv) * XMAT + xr * XROW + xc * 2;
+        uint32_t ah[4], al[4];
+        ldsm_x4_t(xs, ah[0], ah[1], ah[2], ah[3]);
+        ldsm_x4_t(xs + XMAT, al[0], al[1], al[2], al[3]);
+        const uint32_t tile = smem_u32(sm + (size_t)w * TILE * (2 + 2 * kRing)) + kv * TILE;  // Q_w or dO_w
+#pragma unroll
+        for (int jj = 0; jj < NTW; jj += 2) {
+          const int nn = (j0 + jj) >> 1;
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(tile + swz(vrow, 2 * nn + vc), b0, b1, b2, b3);
+          mma_bf16(acc[jj], ah, b0, b1);
+          mma_bf16(acc[jj + 1], ah, b2, b3);
+          mma_bf16(acc[jj], al, b0, b1);
+          mma_bf16(acc[jj + 1], al, b2, b3);
+        }
+      }
+      const float f = (kv == 0) ? p.scale : 1.f;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int ck_idx = ct * 16 + g + 8 * half;
+        if (ck_idx < nc) {
+          const int l = clist[ck_idx] >> 24;
+          float* part = p.part[l] + ((((size_t)bh * NG + grp) * K + cslot[ck_idx]) * 2 + kv) * D;
+#pragma unroll
+          for (int j = 0; j < NTW; ++j)
+            *reinterpret_cast<float2*>(part + 8 * (j0 + j) + 2 * t) =
+                make_float2(acc[j][2 * half] * f, acc[j][2 * half + 1] * f);
+        }
+      }
     }
-    __syncthreads();
+    __syncthreads();  // the exchange matrices are rewritten by the next coarse tile
   }
 
   if (active) {
@@ -428,12 +448,12 @@ bwd_kv_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
   constexpr int HALVES = D / 64;
   constexpr int SIDE = 128;       // LSE[16] and Delta[16] of a stage's query block (fp32)
   constexpr int CROW = 2 * D * 4;  // one coarse gradient row dK(l) | dV(l), fp32
-  // K_c | V_c | kRing x (Q | dO) tiles (each 1024-byte aligned for the
-  // 128-byte swizzle), kRing side buffers, two sets of L-1 coarse rows
+  // K_c | V_c | kRingKV x (Q | dO) tiles (each 1024-byte aligned for the
+  // 128-byte swizzle), kRingKV side buffers, two sets of L-1 coarse rows
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  __shared__ __align__(8) uint64_t bars[1 + kRing];  // [0]: K/V + coarse rows; then the ring
+  __shared__ __align__(8) uint64_t bars[1 + kRingKV];  // [0]: K/V + coarse rows; then the ring
   const int lane = threadIdx.x;
   const int g = lane >> 2, t = lane & 3;
   const int n1 = p.N >> 4;
@@ -444,14 +464,14 @@ bwd_kv_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
   const uint32_t kt = w0, vt = w0 + TILE;
   auto ring_q = [&](int st) { return w0 + (uint32_t)(2 + 2 * st) * TILE; };
   auto ring_do = [&](int st) { return w0 + (uint32_t)(3 + 2 * st) * TILE; };
-  unsigned char* sideb = sm + (2 + 2 * kRing) * TILE;
+  unsigned char* sideb = sm + (2 + 2 * kRingKV) * TILE;
   const uint32_t side0 = smem_u32(sideb);
-  unsigned char* cgb = sideb + kRing * SIDE;
+  unsigned char* cgb = sideb + kRingKV * SIDE;
   const uint32_t kvbar = smem_u32(&bars[0]);
-  auto bar_of = [&](uint32_t pos) { return smem_u32(&bars[1 + pos % kRing]); };
-  auto par_of = [&](uint32_t pos) { return (pos / kRing) & 1u; };
+  auto bar_of = [&](uint32_t pos) { return smem_u32(&bars[1 + pos % kRingKV]); };
+  auto par_of = [&](uint32_t pos) { return (pos / kRingKV) & 1u; };
   if (lane == 0) {
-    for (int i = 0; i <= kRing; ++i) mbar_init(smem_u32(&bars[i]), 1);
+    for (int i = 0; i <= kRingKV; ++i) mbar_init(smem_u32(&bars[i]), 1);
     fence_mbar_init();
   }
   __syncwarp();
@@ -482,7 +502,7 @@ bwd_kv_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
     if ((r >> 5) != R.win) row_window(R, r >> 5);
     const int qb = __shfl_sync(0xffffffffu, R.colw, r & 31);
     if (lane == 0) {
-      const uint32_t st = pos % kRing;
+      const uint32_t st = pos % kRingKV;
       const uint32_t bar = bar_of(pos);
       mbar_arrive_expect_tx(bar, 2u * TILE + SIDE);
       const size_t row0 = (size_t)R.bh * p.N + (size_t)qb * 16;
@@ -531,7 +551,7 @@ bwd_kv_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
   if (cur.item < items) {
     issue_kv(cur, par);
     kv_pending = true;
-    for (int r = 0; r < cur.nq && r < kRing; ++r) issue(cur, r, issued++);
+    for (int r = 0; r < cur.nq && r < kRingKV; ++r) issue(cur, r, issued++);
   }
   const float sc2 = p.scale * kLog2e;
   bool ok = true;
@@ -557,8 +577,8 @@ bwd_kv_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
     if (nq > 0) {
       ok = mbar_wait_bounded(bar_of(pos), par_of(pos));
       if (!ok) break;
-      qk_tile_ss<D>(kt, ring_q(pos % kRing), lane, s_cur);
-      qk_tile_ss<D>(vt, ring_do(pos % kRing), lane, d_cur);
+      qk_tile_ss<D>(kt, ring_q(pos % kRingKV), lane, s_cur);
+      qk_tile_ss<D>(vt, ring_do(pos % kRingKV), lane, d_cur);
     }
     if (nxt.item < items) row_window(nxt, 0);  // its query blocks, for the first issues below
     for (int r = 0; r < nq; ++r) {
@@ -567,29 +587,41 @@ bwd_kv_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
       if (r + 1 < nq) {
         ok = mbar_wait_bounded(bar_of(pr + 1), par_of(pr + 1));
         if (!ok) break;
-        qk_tile_ss<D>(kt, ring_q((pr + 1) % kRing), lane, s_nx);
-        qk_tile_ss<D>(vt, ring_do((pr + 1) % kRing), lane, d_nx);
+        qk_tile_ss<D>(kt, ring_q((pr + 1) % kRingKV), lane, s_nx);
+        qk_tile_ss<D>(vt, ring_do((pr + 1) % kRingKV), lane, d_nx);
       }
-      // LSE and Delta of the queries in this thread's columns: 2t, 2t+1, 8+2t, 9+2t
-      const float* side = reinterpret_cast<const float*>(sideb + (pr % kRing) * SIDE);
+      // LSE and Delta of the queries in this thread's columns 8nt + 2t + j;
+      // pairs of columns run as packed f32x2 operations.  A query without
+      // keys (LSE = -inf) gets exponent -inf, so P = 0.
+      const float* side = reinterpret_cast<const float*>(sideb + (pr % kRingKV) * SIDE);
       float P[2][4], dS[2][4];
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+      for (int nt = 0; nt < 2; ++nt) {
+        const float2 lse = *reinterpret_cast<const float2*>(side + 8 * nt + 2 * t);
+        const float2 del = *reinterpret_cast<const float2*>(side + 16 + 8 * nt + 2 * t);
+        const float a0 = lse.x * kLog2e, a1 = lse.y * kLog2e;
+        const uint64_t nl = f2_make(a0 == -INFINITY ? -INFINITY : -a0, a1 == -INFINITY ? -INFINITY : -a1);
+        const uint64_t dl = f2_make(del.x, del.y);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int qi = 8 * nt + 2 * t + (e & 1);
-          const float l2 = side[qi] * kLog2e;
-          P[nt][e] = (l2 == -INFINITY) ? 0.f : ex2_approx(fmaf(s_cur[nt][e], sc2, -l2));
-          dS[nt][e] = P[nt][e] * (d_cur[nt][e] - side[16 + qi]);
+        for (int h = 0; h < 2; ++h) {  // h = 0: row g (e = 0, 1); h = 1: row g + 8 (e = 2, 3)
+          const float2 x =
+              f2_split(f2_fma(f2_make(s_cur[nt][2 * h], s_cur[nt][2 * h + 1]), f2_make(sc2, sc2), nl));
+          P[nt][2 * h] = ex2_approx(x.x);
+          P[nt][2 * h + 1] = ex2_approx(x.y);
+          const float2 ds = f2_split(f2_mul(f2_make(P[nt][2 * h], P[nt][2 * h + 1]),
+                                            f2_sub(f2_make(d_cur[nt][2 * h], d_cur[nt][2 * h + 1]), dl)));
+          dS[nt][2 * h] = ds.x;
+          dS[nt][2 * h + 1] = ds.y;
         }
+      }
       uint32_t ph[4], pl[4], dsh[4], dsl[4];
       split_frag(P, ph, pl);
       split_frag(dS, dsh, dsl);
-      pv_tile2<D>(ph, pl, ring_do(pr % kRing), lane, dv);
-      pv_tile2<D>(dsh, dsl, ring_q(pr % kRing), lane, dk);
+      pv_tile2<D>(ph, pl, ring_do(pr % kRingKV), lane, dv);
+      pv_tile2<D>(dsh, dsl, ring_q(pr % kRingKV), lane, dk);
       __syncwarp();
       fence_proxy_async_smem();
-      if (r + kRing < nq) issue(cur, r + kRing, issued++);
+      if (r + kRingKV < nq) issue(cur, r + kRingKV, issued++);
       if (r + 1 < nq) {
 #pragma unroll
         for (int a = 0; a < 2; ++a)
@@ -608,7 +640,7 @@ bwd_kv_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant_
     if (nxt.item < items) {
       issue_kv(nxt, par ^ 1);
       kv_pending = true;
-      for (int r = 0; r < nxt.nq && r < kRing; ++r) issue(nxt, r, issued++);
+      for (int r = 0; r < nxt.nq && r < kRingKV; ++r) issue(nxt, r, issued++);
     }
     // epilogue: dK = scale * acc + sum_l coarse dK(l)[t >> 4l] / 16^l (likewise dV)
     bf16* dK = static_cast<bf16*>(p.dk);
@@ -666,7 +698,7 @@ cudaError_t launch_typed(const AttnParams& p, const CUtensorMap* maps, cudaStrea
   e = launch_coarse_reduce(p, s);
   if (e != cudaSuccess) return e;
   // pass 3: persistent single-warp CTAs, as many as fit at once
-  const size_t smem3 = 1024 + (size_t)2 * TILE * (1 + kRing) + kRing * 128 +
+  const size_t smem3 = 1024 + (size_t)2 * TILE * (1 + kRingKV) + kRingKV * 128 +
                        (size_t)2 * (p.L - 1) * 2 * D * sizeof(float);
   e = cudaFuncSetAttribute(bwd_kv_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3);
   if (e != cudaSuccess) return e;

@@ -28,7 +28,10 @@ namespace {
 
 constexpr int kFwdWarps = 4;  // warps per CTA
 constexpr int kBPW = 4;       // consecutive query blocks per warp (same coarse keys)
-constexpr int kStages = 2;
+#ifndef LLSA_FWD_STAGES
+#define LLSA_FWD_STAGES 2
+#endif
+constexpr int kStages = LLSA_FWD_STAGES;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
@@ -52,13 +55,18 @@ template <int NT>
 __device__ __forceinline__ void softmax_tile(float (&s)[2][4], const float (&lw)[2][2], float sc2,
                                              SoftmaxState& st, float (&o)[NT][4],
                                              uint32_t (&pa)[4]) {
+  // pairs of columns run as packed f32x2 operations (bit-identical to scalar)
   float x[2][4];
+  const uint64_t sc2x2 = f2_make(sc2, sc2);
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt) {
-    x[nt][0] = fmaf(s[nt][0], sc2, lw[nt][0]);
-    x[nt][1] = fmaf(s[nt][1], sc2, lw[nt][1]);
-    x[nt][2] = fmaf(s[nt][2], sc2, lw[nt][0]);
-    x[nt][3] = fmaf(s[nt][3], sc2, lw[nt][1]);
+    const uint64_t lwp = f2_make(lw[nt][0], lw[nt][1]);
+    const float2 a = f2_split(f2_fma(f2_make(s[nt][0], s[nt][1]), sc2x2, lwp));
+    const float2 b = f2_split(f2_fma(f2_make(s[nt][2], s[nt][3]), sc2x2, lwp));
+    x[nt][0] = a.x;
+    x[nt][1] = a.y;
+    x[nt][2] = b.x;
+    x[nt][3] = b.y;
   }
   // common path: no max at all, only a check that no score exceeds the
   // reference by more than the threshold (false while the reference is -inf
@@ -83,27 +91,37 @@ __device__ __forceinline__ void softmax_tile(float (&s)[2][4], const float (&lw)
     if (up1) st.m[1] = mx1;
     st.l[0] *= c0;
     st.l[1] *= c1;
+    const uint64_t cc0 = f2_make(c0, c0), cc1 = f2_make(c1, c1);
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      o[nt][0] *= c0;
-      o[nt][1] *= c0;
-      o[nt][2] *= c1;
-      o[nt][3] *= c1;
+      const float2 a = f2_split(f2_mul(f2_make(o[nt][0], o[nt][1]), cc0));
+      const float2 b = f2_split(f2_mul(f2_make(o[nt][2], o[nt][3]), cc1));
+      o[nt][0] = a.x;
+      o[nt][1] = a.y;
+      o[nt][2] = b.x;
+      o[nt][3] = b.y;
     }
   }
   // a row whose every score so far is -inf keeps m = -inf and gets p = 0
   const float b0 = (st.m[0] == -INFINITY) ? 0.f : st.m[0];
   const float b1 = (st.m[1] == -INFINITY) ? 0.f : st.m[1];
   float p[2][4];
+  const uint64_t bb0 = f2_make(b0, b0), bb1 = f2_make(b1, b1);
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt) {
-    p[nt][0] = ex2_approx(x[nt][0] - b0);
-    p[nt][1] = ex2_approx(x[nt][1] - b0);
-    p[nt][2] = ex2_approx(x[nt][2] - b1);
-    p[nt][3] = ex2_approx(x[nt][3] - b1);
+    const float2 a = f2_split(f2_sub(f2_make(x[nt][0], x[nt][1]), bb0));
+    const float2 b = f2_split(f2_sub(f2_make(x[nt][2], x[nt][3]), bb1));
+    p[nt][0] = ex2_approx(a.x);
+    p[nt][1] = ex2_approx(a.y);
+    p[nt][2] = ex2_approx(b.x);
+    p[nt][3] = ex2_approx(b.y);
   }
-  st.l[0] += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
-  st.l[1] += (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]);
+  // l[0] += (p00 + p01) + (p10 + p11), l[1] likewise with p02.., as pairs
+  const uint64_t u = f2_add(f2_make(p[0][0], p[0][2]), f2_make(p[0][1], p[0][3]));
+  const uint64_t v = f2_add(f2_make(p[1][0], p[1][2]), f2_make(p[1][1], p[1][3]));
+  const float2 lsum = f2_split(f2_add(f2_make(st.l[0], st.l[1]), f2_add(u, v)));
+  st.l[0] = lsum.x;
+  st.l[1] = lsum.y;
   pa[0] = pack_bf16(p[0][0], p[0][1]);
   pa[1] = pack_bf16(p[0][2], p[0][3]);
   pa[2] = pack_bf16(p[1][0], p[1][1]);
