@@ -323,7 +323,8 @@ def run_ours(args, rank, world, local_rank):
     host = {k: torch.from_numpy(v).to(dtype=tdt).pin_memory() for k, v in x.items()}
     del x
     desc = llsa.make_desc(w.B, w.H, w.N, w.D, w.L, w.topk, llsa.BF16 if w.dtype == "bf16" else llsa.F32,
-                          flags=llsa.FLAG_FWD_TCGEN05 if args.fwd_tcgen05 else 0)
+                          flags=(llsa.FLAG_FWD_TCGEN05 if args.fwd_tcgen05 else 0)
+                          | (llsa.FLAG_BWD_TCGEN05 if args.bwd_tcgen05 else 0))
     bufs = llsa.LlsaBuffers(desc, dev, with_bwd=w.backward)
     o = torch.empty_like(t_in["q"])
     lse = torch.empty(w.B, w.H, w.N, dtype=torch.float32, device=dev)
@@ -495,6 +496,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true",
                     help="skip the dense scaled_dot_product_attention comparison")
+    ap.add_argument("--bwd-tcgen05", action="store_true",
+                    help="run the key-major backward pass on the tcgen05 kernel (bf16, D=64)")
     ap.add_argument("--fwd-tcgen05", action="store_true",
                     help="run the forward on the tcgen05 kernel (bf16, D=64)")
     args = ap.parse_args()

@@ -28,6 +28,7 @@ F32, BF16 = 0, 1
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_LAUNCH, ERR_WORKSPACE = 0, 1, 2, 3, 4
 DEV_BAD_INDEX, DEV_NONCANONICAL, DEV_TIMEOUT = 1, 2, 4
 FLAG_FWD_TCGEN05 = 1
+FLAG_BWD_TCGEN05 = 2
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 EXPORTED = (

@@ -14,7 +14,7 @@ cudaError_t launch_attn_fwd_simt(const AttnParams& p, int dtype, cudaStream_t s)
 cudaError_t launch_attn_bwd_simt(const AttnParams& p, int dtype, cudaStream_t s);
 cudaError_t launch_attn_fwd_mma(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s);
 cudaError_t launch_attn_fwd_tc(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s);
-cudaError_t launch_attn_bwd_mma(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s);
+cudaError_t launch_attn_bwd_mma(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s, bool tc_kv);
 }  // namespace llsa
 
 using namespace llsa;
@@ -24,12 +24,14 @@ namespace {
 // The tcgen05 forward (attn_fwd_tc.cu) is the bf16 D = 64 default only when
 // it is the faster of the two; LLSA_FLAG_FWD_TCGEN05 selects it explicitly.
 constexpr bool kUseTcForward = false;
+// Likewise for the key-major backward pass; LLSA_FLAG_BWD_TCGEN05 selects it.
+constexpr bool kUseTcBackward = false;
 
 inline int check_desc(const llsa_desc* d) {
   if (d == nullptr) return LLSA_ERR_INVALID_ARG;
   if (d->B < 1 || d->H < 1 || d->N < kBlock || d->D < 1 || d->L < 1 || d->topk < 1)
     return LLSA_ERR_INVALID_ARG;
-  if ((d->flags & ~LLSA_FLAG_FWD_TCGEN05) != 0) return LLSA_ERR_INVALID_ARG;
+  if ((d->flags & ~(LLSA_FLAG_FWD_TCGEN05 | LLSA_FLAG_BWD_TCGEN05)) != 0) return LLSA_ERR_INVALID_ARG;
   if (d->dtype != LLSA_F32 && d->dtype != LLSA_BF16) return LLSA_ERR_INVALID_ARG;
   if (d->D != 64 && d->D != 128) return LLSA_ERR_UNSUPPORTED;
   if (d->L > kMaxL || d->topk > kMaxK) return LLSA_ERR_UNSUPPORTED;
@@ -359,7 +361,8 @@ int llsa_attn_bwd(const llsa_desc* desc, const void* q, const void* k, const voi
     st = make_row_tile_map(&maps[i], srcs[i], rows, desc->D);
     if (st != LLSA_OK) return st;
   }
-  return launch_status(launch_attn_bwd_mma(p, maps, (cudaStream_t)stream));
+  const bool tc_kv = kUseTcBackward || (desc->flags & LLSA_FLAG_BWD_TCGEN05) != 0;
+  return launch_status(launch_attn_bwd_mma(p, maps, (cudaStream_t)stream, tc_kv));
 }
 
 }  // extern "C"

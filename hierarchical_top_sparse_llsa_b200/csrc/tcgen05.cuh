@@ -108,11 +108,13 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
 }
 
 // Instruction descriptor of kind::f16 with bf16 A and B, f32 accumulation,
-// M x N tile; b_mn_major selects an MN-major B operand (A is K-major).
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int b_mn_major) {
+// M x N tile; b_mn_major / a_mn_major select MN-major operands (otherwise
+// K-major).
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int b_mn_major, int a_mn_major = 0) {
   return (1u << 4)                        // D format: f32
          | (1u << 7)                      // A format: bf16
          | (1u << 10)                     // B format: bf16
+         | ((uint32_t)a_mn_major << 15)   // A major
          | ((uint32_t)b_mn_major << 16)   // B major
          | ((uint32_t)(N >> 3) << 17)     // N / 8
          | ((uint32_t)(M >> 4) << 24);    // M / 16

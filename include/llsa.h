@@ -66,7 +66,11 @@ enum {
   /* bf16, D = 64: run llsa_attn_fwd on the tcgen05 kernel (tensor-memory
    * accumulators, 8 sibling query blocks per 128-row MMA) instead of the
    * warp-MMA kernel.  Both compute the same result within bf16 rounding. */
-  LLSA_FLAG_FWD_TCGEN05 = 1
+  LLSA_FLAG_FWD_TCGEN05 = 1,
+  /* bf16, D = 64: run the key-major pass of llsa_attn_bwd (dK, dV) on the
+   * tcgen05 kernel (8 query blocks of a key block per 128-row MMA, dK and dV
+   * accumulated in tensor memory) instead of the warp-MMA kernel. */
+  LLSA_FLAG_BWD_TCGEN05 = 2
 };
 
 /* device status bits (OR-ed into *dev_status) */

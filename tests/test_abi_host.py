@@ -57,7 +57,7 @@ def _desc(**kw):
     (dict(topk=0), llsa.ERR_INVALID_ARG),
     (dict(dtype=5), llsa.ERR_INVALID_ARG),
     (dict(B=0), llsa.ERR_INVALID_ARG),
-    (dict(flags=2), llsa.ERR_INVALID_ARG),
+    (dict(flags=4), llsa.ERR_INVALID_ARG),
 ])
 def test_bad_descriptors_are_rejected_before_launch(lib, kw, status):
     d = _desc(**kw)

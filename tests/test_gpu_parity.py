@@ -198,3 +198,44 @@ def test_forward_external_indices_and_weights(flags):
     r = run_oracle(x, L, K, idx=clean, bwd=False, level_w=lw)
     assert_close(g["O"], r["O"], "bf16", "O")
     assert_close(g["LSE"], r["LSE"], "bf16", "LSE")
+
+
+@pytest.mark.parametrize("name,heads", [
+    ("img64_bf16", None),
+    ("img128_bf16", [0, 11]),
+    ("img256_bf16", [5]),
+])
+def test_tcgen05_backward(name, heads):
+    # the tcgen05 key-major backward pass, selected by LLSA_FLAG_BWD_TCGEN05
+    w = workloads.WORKLOADS[name]
+    x = workloads.make_inputs(w)
+    g = run_gpu(w.B, w.H, w.N, w.D, w.L, w.topk, w.dtype, x, flags=llsa.FLAG_BWD_TCGEN05)
+    assert g["status"] == 0
+    hs = slice(None) if heads is None else heads
+    xs = x if heads is None else {k: np.ascontiguousarray(v[:, heads]) for k, v in x.items()}
+    r = run_oracle(xs, w.L, w.topk)
+    _compare(w, g, r, hs, True)
+
+
+def test_tcgen05_backward_external_indices_and_long_rows():
+    # caller indices with skipped entries, empty rows and one key block kept by
+    # every query block (a key-major row of 256 query blocks: 32 groups)
+    B, H, N, D, L, K = 1, 2, 4096, 64, 3, 6
+    x = _small(29, B, H, N, D)
+    rng = np.random.default_rng(30)
+    ext = {}
+    for l in range(1, L + 1):
+        n = N // 16**l
+        I = rng.integers(-3, n + 3, size=(B, H, n, K)).astype(np.int32)
+        I[..., 0, :] = -1
+        ext[l] = I
+    ext[1][0, 1, :, 0] = 7
+    ext[1][0, 1, :, 1:] = np.sort(rng.choice(np.arange(8, 256), size=(256, K - 1), replace=True), axis=1)
+    clean = {}
+    for l in range(1, L + 1):
+        clean[l], _ = clean_indices(ext[l], N // 16**l)
+    lw = [0, 0, 16.0**2, 16.0**3]
+    g = run_gpu(B, H, N, D, L, K, "bf16", x, ext_idx=ext, level_w=lw, flags=llsa.FLAG_BWD_TCGEN05)
+    r = run_oracle(x, L, K, idx=clean, level_w=lw)
+    for name in ("dQ", "dK", "dV"):
+        assert_close(g[name], r[name], "bf16", name)
