@@ -110,7 +110,10 @@ def committed_traffic(workload: str, stage: str):
     m = re.search(r"```json\n(.*?)\n```", text, re.S)
     if m is None:
         return None
-    rec = json.loads(m.group(1))
+    try:
+        rec = json.loads(m.group(1))
+    except ValueError:
+        return None
     if rec.get("sources_sha1") != sources_digest():
         return None
     st = rec.get("stages", {}).get(stage)
