@@ -336,7 +336,7 @@ def run_ours(args, rank, world, local_rank):
     sh = stream.cuda_stream
     st = bufs.status.data_ptr()
 
-    def step(tin, ev=None):
+    def step(tin, ev=None, sh=sh):
         q, k, v = tin["q"].data_ptr(), tin["k"].data_ptr(), tin["v"].data_ptr()
         if ev is not None:
             ev[0].record(stream)
@@ -370,6 +370,25 @@ def run_ours(args, rank, world, local_rank):
     if int(bufs.status.item()) != 0:
         raise RuntimeError(f"device status {int(bufs.status.item())} during warm-up")
 
+    # the whole step as one CUDA graph (its 15 launches replayed without host
+    # round trips or launch gaps); the per-stage breakdown below comes from
+    # a separate loop of direct calls with events between the stages
+    graph, graph_note = None, "disabled (--no-graph)"
+    if not args.no_graph:
+        try:
+            g = torch.cuda.CUDAGraph()
+            cs = torch.cuda.Stream(dev)
+            cs.wait_stream(stream)
+            with torch.cuda.graph(g, stream=cs):
+                step(t_in, None, cs.cuda_stream)
+            stream.wait_stream(cs)
+            g.replay()
+            torch.cuda.synchronize()
+            graph, graph_note = g, "captured"
+        except RuntimeError as exc:  # capture refused: time direct calls instead
+            torch.cuda.synchronize()
+            graph_note = f"not captured ({str(exc).splitlines()[0][:120]})"
+
     nst = 6 if w.backward else 4
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nst)] for _ in range(args.steps)]
     barrier()
@@ -381,13 +400,20 @@ def run_ours(args, rank, world, local_rank):
     t_end = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
     for s in range(args.steps):
-        step(t_in, evs[s])
+        if graph is not None:
+            graph.replay()
+        else:
+            step(t_in, evs[s])
     t_end.record(stream)
     torch.cuda.synchronize()
     barrier()
     if sampler:
         sampler.__exit__()
     ms = t_start.elapsed_time(t_end) / args.steps
+    if graph is not None:  # stage breakdown from direct calls
+        for s in range(args.steps):
+            step(t_in, evs[s])
+        torch.cuda.synchronize()
     stage_ms = {}
     names = STAGES if w.backward else STAGES[:3]
     for i, name in enumerate(names):
@@ -484,6 +510,7 @@ def run_ours(args, rank, world, local_rank):
         "e2e": {"value": world * tokens / (e2e_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": nlaunch * args.steps,
+        "cuda_graph": graph_note,
         "clocks": sampler.summary() if sampler else None,
     }
     print(json.dumps(line), flush=True)
@@ -497,6 +524,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=workloads.HEADLINE, choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time direct calls instead of a CUDA graph of the step")
     ap.add_argument("--no-dense", action="store_true",
                     help="skip the dense scaled_dot_product_attention comparison")
     ap.add_argument("--bwd-tcgen05", action="store_true",
