@@ -689,6 +689,8 @@ cudaError_t launch_typed(const AttnParams& p, const CUtensorMap* maps, cudaStrea
                        nct * 16 * sizeof(float) + kQWarps * (1 + kRing) * 8 + 2 * nct * 16 * sizeof(int);
   cudaError_t e = cudaFuncSetAttribute(bwd_q_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
   if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(bwd_q_mma_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
   bwd_q_mma_kernel<D><<<dim3((n1 + kQWarps - 1) / kQWarps, BH), kQWarps * 32, smem1, s>>>(
       maps[0], maps[1], maps[2], maps[3], p, nct);
   e = cudaGetLastError();

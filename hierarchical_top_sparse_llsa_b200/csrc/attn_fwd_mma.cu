@@ -361,6 +361,8 @@ cudaError_t launch_typed(const AttnParams& p, const CUtensorMap* maps, cudaStrea
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_mma_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(attn_fwd_mma_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+  if (e != cudaSuccess) return e;
   const int n1 = p.N / kBlock;
   const int per_cta = kFwdWarps * kBPW;
   dim3 grid((n1 + per_cta - 1) / per_cta, p.B * p.H);

@@ -76,8 +76,8 @@ select_kernel(SelectParams p) {
   extern __shared__ float4 smem4[];
   float* qsT = reinterpret_cast<float*>(smem4);   // [D][16] queries, transposed
   float* ksT = qsT + D * QLD;                     // [D][CLD] candidates, transposed
-  float* sc = ksT + D * CLD;                      // [16][kSelChunk] scores of a chunk
-  int* cid = reinterpret_cast<int*>(sc + kSelQ * kSelChunk);  // [kSelChunk]
+  float* sc = ksT;                                // [16][kSelChunk] scores of a chunk (over ksT)
+  int* cid = reinterpret_cast<int*>(ksT + D * CLD);  // [kSelChunk]
   __shared__ int parents[kMaxK];
   __shared__ int n_par;
 
@@ -169,6 +169,7 @@ select_kernel(SelectParams p) {
         acc[a][1] = (d == 0) ? m23 : f2_add(acc[a][1], m23);
       }
     }
+    __syncthreads();  // every thread is done with ksT, which the scores overwrite
 #pragma unroll
     for (int a = 0; a < 4; ++a) {
       float4 o;
@@ -238,10 +239,12 @@ select_kernel(SelectParams p) {
 
 template <int D>
 cudaError_t launch_sel(const SelectParams& p, int BH, cudaStream_t s) {
-  const size_t smem = (size_t)(D * kSelQ + D * (kSelChunk + 4) + kSelQ * kSelChunk) * sizeof(float) +
-                      kSelChunk * sizeof(int);
+  static_assert(kSelQ * kSelChunk <= 64 * (kSelChunk + 4), "scores fit over the candidate tile");
+  const size_t smem = (size_t)(D * kSelQ + D * (kSelChunk + 4)) * sizeof(float) + kSelChunk * sizeof(int);
   // set on every call: the attribute is per device and the call is cheap
   cudaError_t e = cudaFuncSetAttribute(select_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(select_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   const int groups = (p.parent == nullptr) ? (p.n + kSelQ - 1) / kSelQ : p.n / kBlock;
   select_kernel<D><<<dim3(groups, BH), kSelThreads, smem, s>>>(p);
