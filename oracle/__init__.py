@@ -24,10 +24,14 @@ Parity status of each function (what pins it, in tests/test_oracle_*.py):
   index_transpose  pinned: dense block-mask transpose, pair-count invariants,
                    the 100-query x 8-key example (800 pairs).
   attn_bwd         pinned: central finite differences of <dO, O>.
+  zorder_index     pinned: the 4x4 grid written out by hand, a decoded
+  reorder          token, 4x4-tile runs, round trips.
 """
 
 from .llsa_oracle import (  # noqa: F401
     pool,
+    reorder,
+    zorder_index,
     select_level,
     select_all,
     candidates_for_level,

@@ -372,3 +372,39 @@ def run_forward(Q, K, V, L, topk, scale=None, level_w=None):
     idx = select_all(pq, pk, L, topk)
     O, LSE = attn_fwd(Q, K, V, pk, pv, idx, L, scale, level_w)
     return {"pq": pq, "pk": pk, "pv": pv, "idx": idx, "O": O, "LSE": LSE, "scale": scale}
+
+
+# --------------------------------------------------------------------------
+# Step 5: index reordering for images (raster <-> Z-order)
+# --------------------------------------------------------------------------
+def zorder_index(img_h: int, img_w: int) -> np.ndarray:
+    """Z-order token of every raster position y * img_w + x (Step 5, Index
+    Reordering for Images: group 2x2 pixels, then 4x4, ...).  The Z-order
+    index interleaves the bits of x and y, x taking the even bits and y the
+    odd bits, so 4 consecutive tokens are a 2x2 tile, 16 a 4x4 tile and so
+    on.  Reading taken: square images whose side is a power of two (the
+    pages' images are square); other shapes are rejected."""
+    if img_h != img_w or img_h < 1 or (img_h & (img_h - 1)) != 0:
+        raise ValueError("square power-of-two images only")
+    z = np.zeros(img_h * img_w, dtype=np.int64)
+    bits = img_w.bit_length() - 1
+    for y in range(img_h):
+        for x in range(img_w):
+            t = 0
+            for b in range(bits):
+                t |= ((x >> b) & 1) << (2 * b)
+                t |= ((y >> b) & 1) << (2 * b + 1)
+            z[y * img_w + x] = t
+    return z
+
+
+def reorder(X: np.ndarray, img_h: int, img_w: int, to_zorder: bool) -> np.ndarray:
+    """Permute the token axis of X [B, H, N, D] between raster order
+    (y * img_w + x) and Z-order (zorder_index); a pure permutation."""
+    z = zorder_index(img_h, img_w)
+    out = np.empty_like(X)
+    if to_zorder:
+        out[:, :, z, :] = X
+    else:
+        out[:, :, :, :] = X[:, :, z, :]
+    return out
