@@ -168,6 +168,32 @@ def max_over_ranks(torch, dist, values, device) -> list:
     return [float(x) for x in t.tolist()]
 
 
+def reorder_rate(torch, llsa, w, dev, src, hbm_gbs, iters=10):
+    """Raster -> Z-order permutation of one [B, H, N, D] tensor (llsa_reorder,
+    for callers that hold raster-order tokens): ms per call and GB/s of its
+    compulsory traffic (read + write once).  Not part of the step."""
+    side = int(round(w.N ** 0.5))
+    if side * side != w.N:
+        return None
+    dst = torch.empty_like(src)
+    sh = torch.cuda.current_stream(dev).cuda_stream
+    dt = llsa.BF16 if src.dtype == torch.bfloat16 else llsa.F32
+    call = lambda: llsa.llsa_reorder(w.B, w.H, side, side, w.D, dt, src.data_ptr(), dst.data_ptr(), True, sh)
+    call()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(iters):
+        call()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / iters
+    gbs = 2 * src.numel() * src.element_size() / (ms * 1e-3) / 1e9
+    return {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm_gbs, 4),
+            "tensor": f"[{w.B}, {w.H}, {w.N}, {w.D}] {str(src.dtype).replace('torch.', '')}"}
+
+
 def launches_per_step(L: int) -> dict:
     """Kernels each entry point launches (matches the C library's dispatch)."""
     return {"pool": 1 + max(0, L - 2), "select": L, "fwd": 1, "transpose": 4,
@@ -484,6 +510,7 @@ def run_ours(args, rank, world, local_rank):
                               "null: no ncu capture of the current sources")
     roof["kernel"] = f"llsa_{'attn_' if dom in ('fwd', 'bwd') else ''}{dom} ({launches_per_step(w.L)[dom]} launches)"
     roof["peak_source"] = f"{peaks['source']} (MEASURED_PEAKS.json)" if peaks["source"] == "measured" else "fallback"
+    reorder = reorder_rate(torch, llsa, w, dev, t_in["q"], peaks["hbm_gbs"])
     dense = None
     if w.backward and not args.no_dense:
         dense = dense_reference(torch, w, dev)
@@ -507,6 +534,7 @@ def run_ours(args, rank, world, local_rank):
         "roofline": roof,
         "cpu_baseline": cpu,
         "dense_reference": dense,
+        "reorder": reorder,
         "e2e": {"value": world * tokens / (e2e_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": nlaunch * args.steps,

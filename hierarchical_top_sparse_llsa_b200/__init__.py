@@ -40,6 +40,7 @@ EXPORTED = (
     "llsa_bwd_workspace_bytes",
     "llsa_attn_bwd",
     "llsa_attn_bwd_noalloc",
+    "llsa_reorder",
     "llsa_status_string",
     "llsa_version",
 )
@@ -98,6 +99,8 @@ def lib() -> ctypes.CDLL:
                                              vp, vp]),
             "llsa_attn_bwd_noalloc": (ctypes.c_int, [P(LlsaDesc), vp, vp, vp, P(LlsaPyramid), vp, vp, vp,
                                                      P(LlsaIndices), P(LlsaCsr), vp, vp, vp, vp, vp]),
+            "llsa_reorder": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                            ctypes.c_int, vp, vp, ctypes.c_int, vp]),
             "llsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
             "llsa_version": (ctypes.c_int, []),
         }
@@ -177,6 +180,12 @@ def llsa_attn_bwd_noalloc(desc, q, k, v, pyramid, o, lse, dout, indices, csr, dq
     st = lib().llsa_attn_bwd_noalloc(ctypes.byref(desc), q, k, v, ctypes.byref(pyramid), o, lse, dout,
                                      ctypes.byref(indices), ctypes.byref(csr), dq, dk, dv, dev_status,
                                      stream)
+    return _check(st) if check else st
+
+
+def llsa_reorder(B, H, img_h, img_w, D, dtype, src, dst, to_zorder, stream=0, check=True):
+    """Raster <-> Z-order permutation of the token axis of [B, H, N, D]."""
+    st = lib().llsa_reorder(B, H, img_h, img_w, D, dtype, src, dst, 1 if to_zorder else 0, stream)
     return _check(st) if check else st
 
 

@@ -178,6 +178,26 @@ extern "C" {
 
 int llsa_version(void) { return 100; }
 
+int llsa_reorder(int B, int H, int img_h, int img_w, int D, int dtype, const void* src, void* dst,
+                 int to_zorder, void* stream) {
+  if (B < 1 || H < 1 || img_h < 1 || img_w < 1 || src == nullptr || dst == nullptr) return LLSA_ERR_INVALID_ARG;
+  if (dtype != LLSA_F32 && dtype != LLSA_BF16) return LLSA_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return LLSA_ERR_UNSUPPORTED;
+  if (img_h != img_w || img_h < 4 || (img_h & (img_h - 1)) != 0 || img_h > (1 << 15)) return LLSA_ERR_UNSUPPORTED;
+  if ((((uintptr_t)src | (uintptr_t)dst) & 15) != 0) return LLSA_ERR_INVALID_ARG;
+  const long long N = (long long)img_h * img_w;
+  const long long rows = (long long)B * H * N;
+  const int row_bytes = D * (dtype == LLSA_BF16 ? 2 : 4);
+  const uintptr_t bytes = (uintptr_t)(rows * row_bytes);
+  const uintptr_t a = (uintptr_t)src, b = (uintptr_t)dst;
+  if (a < b + bytes && b < a + bytes) return LLSA_ERR_INVALID_ARG;  // overlapping buffers
+  if (N > 0x7fffffffLL) return LLSA_ERR_UNSUPPORTED;
+  int side_log2 = 0;
+  while ((1 << side_log2) < img_w) ++side_log2;
+  return launch_status(launch_reorder(src, dst, rows, (int)N, side_log2, row_bytes, to_zorder != 0,
+                                      (cudaStream_t)stream));
+}
+
 const char* llsa_status_string(int status) {
   switch (status) {
     case LLSA_OK: return "ok";

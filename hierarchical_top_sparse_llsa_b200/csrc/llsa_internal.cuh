@@ -184,5 +184,7 @@ cudaError_t launch_transpose(const TransposeParams& p, cudaStream_t s);
 void transpose_chunking(int n, int* nchunk, int* rows);
 int transpose_prefix_tiles(int n);
 cudaError_t launch_coarse_reduce(const AttnParams& p, cudaStream_t s);
+cudaError_t launch_reorder(const void* src, void* dst, long long rows, int N, int side_log2, int row_bytes,
+                           int to_zorder, cudaStream_t s);
 
 }  // namespace llsa

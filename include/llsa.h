@@ -243,6 +243,22 @@ LLSA_API int llsa_attn_bwd_noalloc(const llsa_desc* desc, const void* q, const v
                                    const llsa_csr* csr, void* dq, void* dk, void* dv,
                                    int32_t* dev_status, void* stream);
 
+/*
+ * llsa_reorder - raster <-> Z-order permutation of the token axis (Step 5:
+ * Index Reordering for Images), for callers whose tokens are in raster order
+ * (token y * img_w + x for pixel (x, y)).  Z-order token t holds the pixel
+ * whose x is made of the even bits of t and whose y of the odd bits, so 16
+ * consecutive tokens form a 4x4 tile (the layout every other call expects).
+ *   B, H: batch and heads; img_h == img_w, a power of two >= 4 (N = img_h *
+ *   img_w tokens; other shapes give LLSA_ERR_UNSUPPORTED); D in {64, 128};
+ *   dtype: LLSA_F32 or LLSA_BF16.
+ *   src, dst: [B, H, N, D] device tensors of dtype, 16-byte aligned, not
+ *   overlapping (overlap gives LLSA_ERR_INVALID_ARG).
+ *   to_zorder: nonzero for raster -> Z-order, 0 for Z-order -> raster.
+ */
+LLSA_API int llsa_reorder(int B, int H, int img_h, int img_w, int D, int dtype, const void* src, void* dst,
+                          int to_zorder, void* stream);
+
 /* Static text for a host status code. */
 LLSA_API const char* llsa_status_string(int status);
 

@@ -135,3 +135,21 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(llsa, "_lib", None)
     with pytest.raises(llsa.LlsaError):
         llsa.lib()
+
+
+@pytest.mark.parametrize("args,status", [
+    (dict(img_h=8, img_w=16), llsa.ERR_UNSUPPORTED),   # not square
+    (dict(img_h=12, img_w=12), llsa.ERR_UNSUPPORTED),  # not a power of two
+    (dict(img_h=2, img_w=2), llsa.ERR_UNSUPPORTED),    # smaller than a 4x4 tile
+    (dict(D=96), llsa.ERR_UNSUPPORTED),
+    (dict(dtype=7), llsa.ERR_INVALID_ARG),
+    (dict(B=0), llsa.ERR_INVALID_ARG),
+    (dict(src=None), llsa.ERR_INVALID_ARG),
+    (dict(src=1 << 20, dst=(1 << 20) + 1024), llsa.ERR_INVALID_ARG),  # overlapping
+    (dict(src=(1 << 20) + 8), llsa.ERR_INVALID_ARG),                  # not 16-byte aligned
+])
+def test_reorder_argument_checks(lib, args, status):
+    a = dict(B=1, H=2, img_h=16, img_w=16, D=64, dtype=llsa.BF16, src=1 << 20, dst=1 << 30)
+    a.update(args)
+    assert llsa.llsa_reorder(a["B"], a["H"], a["img_h"], a["img_w"], a["D"], a["dtype"], a["src"], a["dst"],
+                             True, check=False) == status
