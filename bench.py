@@ -194,6 +194,53 @@ def reorder_rate(torch, llsa, w, dev, src, hbm_gbs, iters=10):
             "tensor": f"[{w.B}, {w.H}, {w.N}, {w.D}] {str(src.dtype).replace('torch.', '')}"}
 
 
+def select_scaling(args):
+    """Selection cost against N: hierarchical (the levels of the path's
+    workloads: L = 3 up to 256x256 pixels, 4 at 512x512) and single-level (L = 1: every query block scores every
+    key block, the prior-art baseline the pages compare with), on the same
+    kernels, B = 1, H = 8, D = 64, K = 8, bf16 inputs of the synthetic
+    image-like recipe.  Prints one JSON line; not part of the step."""
+    import torch
+
+    import hierarchical_top_sparse_llsa_b200 as llsa
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    out = []
+    for side in (64, 128, 256, 512):
+        N = side * side
+        Lh = {64: 3, 128: 3, 256: 3, 512: 4}[side]
+        w = workloads.Workload(f"sel{side}", 1, 8, N, 64, "bf16", Lh, 8, 2000 + side, backward=False)
+        x = workloads.make_inputs(w, with_dout=False)
+        q, k, v = (torch.from_numpy(x[n]).to(dev, dtype=torch.bfloat16) for n in ("q", "k", "v"))
+        rec = {"side": side, "N": N}
+        for L in (Lh, 1):
+            desc = llsa.make_desc(w.B, w.H, N, 64, L, 8, llsa.BF16)
+            bufs = llsa.LlsaBuffers(desc, dev, with_bwd=False)
+            sh = torch.cuda.current_stream(dev).cuda_stream
+            llsa.llsa_pool(desc, q.data_ptr(), k.data_ptr(), v.data_ptr(), bufs.pyramid, sh)
+            llsa.llsa_select(desc, bufs.pyramid, bufs.indices, sh)
+            torch.cuda.synchronize()
+            iters = 5 if L == 1 and side >= 512 else 20
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(iters):
+                llsa.llsa_select(desc, bufs.pyramid, bufs.indices, sh)
+            b.record()
+            torch.cuda.synchronize()
+            rec["hierarchical_ms" if L == Lh else "flat_ms"] = round(a.elapsed_time(b) / iters, 4)
+            if L == Lh:
+                rec["levels"] = Lh
+            del bufs
+        rec["flat_over_hierarchical"] = round(rec["flat_ms"] / rec["hierarchical_ms"], 2)
+        out.append(rec)
+        del q, k, v
+        torch.cuda.empty_cache()
+    print(json.dumps({"select_scaling": out, "B": 1, "H": 8, "D": 64, "topk": 8, "dtype": "bf16",
+                      "data": "synthetic image-like"}), flush=True)
+
+
 def launches_per_step(L: int) -> dict:
     """Kernels each entry point launches (matches the C library's dispatch)."""
     return {"pool": 1 + max(0, L - 2), "select": L, "fwd": 1, "transpose": 4,
@@ -552,6 +599,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=workloads.HEADLINE, choices=sorted(workloads.WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--select-scaling", action="store_true",
+                    help="time hierarchical vs single-level selection against N (separate report)")
     ap.add_argument("--no-graph", action="store_true",
                     help="time direct calls instead of a CUDA graph of the step")
     ap.add_argument("--no-dense", action="store_true",
@@ -568,6 +617,9 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if world != args.gpus:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    if args.select_scaling:
+        select_scaling(args)
+        return
     if args.impl == "reference":
         run_reference(args, rank, world)
         return
