@@ -41,10 +41,9 @@
 
 namespace llsa {
 
-// tcgen05 key-major pass (attn_bwd_tcws.cu, warp-specialised): bf16, D = 64;
-// maps as below
+// tcgen05 key-major pass (attn_bwd_tc.cu): bf16, D = 64; maps as below
 bool bwd_kv_tc_supported(const AttnParams& p);
-cudaError_t launch_bwd_kv_tcws(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s);
+cudaError_t launch_bwd_kv_tc(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s);
 
 namespace {
 
@@ -700,7 +699,7 @@ cudaError_t launch_typed(const AttnParams& p, const CUtensorMap* maps, cudaStrea
   e = launch_coarse_reduce(p, s);
   if (e != cudaSuccess) return e;
   // pass 3 on tcgen05 (D = 64) when asked for
-  if (tc_kv && bwd_kv_tc_supported(p)) return launch_bwd_kv_tcws(p, maps, s);
+  if (tc_kv && bwd_kv_tc_supported(p)) return launch_bwd_kv_tc(p, maps, s);
   // pass 3: persistent single-warp CTAs, as many as fit at once
   const size_t smem3 = 1024 + (size_t)2 * TILE * (1 + kRingKV) + kRingKV * 128 +
                        (size_t)2 * (p.L - 1) * 2 * D * sizeof(float);
