@@ -30,6 +30,7 @@ Parity status of each function (what pins it, in tests/test_oracle_*.py):
 
 from .llsa_oracle import (  # noqa: F401
     pool,
+    enriched_top,
     reorder,
     zorder_index,
     select_level,

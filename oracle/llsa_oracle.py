@@ -168,14 +168,27 @@ def select_all(pyr_q: dict, pyr_k: dict, L: int, topk: int, factor: int = FACTOR
 # --------------------------------------------------------------------------
 # Step 3: sparse attention with hierarchical KV enrichment and reweighting
 # --------------------------------------------------------------------------
-def key_sets(idx: dict, L: int, n_blocks: int):
+def enriched_top(L: int, enrich=None) -> int:
+    """Highest level whose pooled tokens enrich the keys, for an enrichment
+    depth Le (Limitations: "enrichment depth Le"; Surprising Findings: more
+    enrichment levels, a little more quality for a little more time).
+    Reading taken: depth Le uses levels 2..1+Le; None or 0 means every
+    coarse level (2..L), a negative value none."""
+    if enrich is None or enrich == 0:
+        return L
+    if enrich < 0:
+        return 1
+    return min(L, 1 + int(enrich))
+
+
+def key_sets(idx: dict, L: int, n_blocks: int, enrich=None):
     """The key set of every 16-token query block b (Step 3).
 
     Fine part: the 16 fine tokens of every level-1 block in I(1)[b].
-    Coarse part, for each level l = 2..L: the level-l tokens in I(l)[a], where
-    a = b // 16**(l-1) is the level-l ancestor of block b.  Level-1 pooled
-    tokens are never keys (the fine tokens of the selected blocks stand for
-    them).
+    Coarse part, for each level l = 2..Lc (Lc = enriched_top(L, enrich)): the
+    level-l tokens in I(l)[a], where a = b // 16**(l-1) is the level-l
+    ancestor of block b.  Level-1 pooled tokens are never keys (the fine
+    tokens of the selected blocks stand for them).
 
     Returns (fine_tok int64 [B,H,n_blocks,16*K], coarse {l: int64
     [B,H,n_blocks,K]}) with -1 for padding.
@@ -185,7 +198,7 @@ def key_sets(idx: dict, L: int, n_blocks: int):
     fine = np.where(I1[..., None] >= 0, I1[..., None] * FACTOR + j, -1)
     fine = fine.reshape(*I1.shape[:-1], I1.shape[-1] * FACTOR)
     coarse = {}
-    for l in range(2, L + 1):
+    for l in range(2, enriched_top(L, enrich) + 1):
         anc = np.arange(n_blocks) // FACTOR ** (l - 1)
         coarse[l] = np.asarray(idx[l], dtype=np.int64)[:, :, anc, :]
     return fine, coarse
@@ -197,7 +210,7 @@ def _gather_keys(Kbh, Vbh, pk, pv, fine, coarse, L, level_w):
     vs = [Vbh[np.maximum(fine, 0)]]
     lw = [np.zeros(fine.shape)]
     ok = [fine >= 0]
-    for l in range(2, L + 1):
+    for l in sorted(coarse):
         c = coarse[l]
         ks.append(pk[l][np.maximum(c, 0)])
         vs.append(pv[l][np.maximum(c, 0)])
@@ -208,7 +221,7 @@ def _gather_keys(Kbh, Vbh, pk, pv, fine, coarse, L, level_w):
             np.concatenate(lw, axis=1), np.concatenate(ok, axis=1))
 
 
-def attn_fwd(Q, K, V, pyr_k, pyr_v, idx, L, scale, level_w=None, block_chunk=512):
+def attn_fwd(Q, K, V, pyr_k, pyr_v, idx, L, scale, level_w=None, block_chunk=512, enrich=None):
     """Forward of LLSA attention (Step 3), as dense attention over each query
     block's explicit key list, in fp64.
 
@@ -222,11 +235,12 @@ def attn_fwd(Q, K, V, pyr_k, pyr_v, idx, L, scale, level_w=None, block_chunk=512
     O_i = 0 and LSE_i = -inf.
 
     pyr_k, pyr_v: {l: [B,H,N_l,D]} for l = 2..L (any float type).
+    enrich: enrichment depth (enriched_top).
     Returns O float64 [B,H,N,D], LSE float64 [B,H,N].
     """
     B, H, N, D = Q.shape
     nb = N // FACTOR
-    fine, coarse = key_sets(idx, L, nb)
+    fine, coarse = key_sets(idx, L, nb, enrich)
     O = np.zeros((B, H, N, D))
     LSE = np.full((B, H, N), -np.inf)
     for b in range(B):
@@ -289,7 +303,7 @@ def index_transpose(idx_l: np.ndarray, n_keys: int):
 # --------------------------------------------------------------------------
 # Backward of Step 3 (the pass that the transpose serves)
 # --------------------------------------------------------------------------
-def attn_bwd(Q, K, V, pyr_k, pyr_v, O, LSE, dO, idx, L, scale, level_w=None, block_chunk=512):
+def attn_bwd(Q, K, V, pyr_k, pyr_v, O, LSE, dO, idx, L, scale, level_w=None, block_chunk=512, enrich=None):
     """Gradients of the LLSA attention (fp64), with the indices held fixed.
 
     With P_ij = w_j exp(s_ij - LSE_i) on the key set of i's block:
@@ -306,7 +320,7 @@ def attn_bwd(Q, K, V, pyr_k, pyr_v, O, LSE, dO, idx, L, scale, level_w=None, blo
     """
     B, H, N, D = Q.shape
     nb = N // FACTOR
-    fine, coarse = key_sets(idx, L, nb)
+    fine, coarse = key_sets(idx, L, nb, enrich)
     dQ = np.zeros((B, H, N, D))
     dK = np.zeros((B, H, N, D))
     dV = np.zeros((B, H, N, D))
@@ -342,7 +356,7 @@ def attn_bwd(Q, K, V, pyr_k, pyr_v, O, LSE, dO, idx, L, scale, level_w=None, blo
                 np.add.at(dK[b, h], fi[m], dk[:, :nf][m])
                 np.add.at(dV[b, h], fi[m], dv[:, :nf][m])
                 off = nf
-                for l in range(2, L + 1):
+                for l in sorted(co):
                     c = co[l]
                     kk = c.shape[-1]
                     m = c >= 0
