@@ -51,6 +51,7 @@ class LlsaDesc(ctypes.Structure):
         ("B", ctypes.c_int), ("H", ctypes.c_int), ("N", ctypes.c_int), ("D", ctypes.c_int),
         ("L", ctypes.c_int), ("topk", ctypes.c_int), ("dtype", ctypes.c_int), ("flags", ctypes.c_int),
         ("sm_scale", ctypes.c_float), ("level_w", ctypes.c_float * (MAX_LEVELS + 1)),
+        ("enrich_levels", ctypes.c_int),
     ]
 
 
@@ -118,13 +119,18 @@ def _check(status: int) -> int:
     return status
 
 
-def make_desc(B, H, N, D, L, topk, dtype, sm_scale=0.0, level_w=None, flags=0) -> LlsaDesc:
-    """Fill an llsa_desc; level_w is None (every weight 1) or indexable by level."""
+def make_desc(B, H, N, D, L, topk, dtype, sm_scale=0.0, level_w=None, flags=0,
+              enrich_levels=0) -> LlsaDesc:
+    """Fill an llsa_desc; level_w is None (every weight 1) or indexable by level.
+
+    enrich_levels is the enrichment depth: coarse levels 2..min(L, 1 + depth)
+    join the keys; 0 means all of them, a negative value none."""
     d = LlsaDesc()
     d.B, d.H, d.N, d.D, d.L, d.topk = B, H, N, D, L, topk
     d.dtype = dtype
     d.flags = flags
     d.sm_scale = sm_scale
+    d.enrich_levels = int(enrich_levels)
     for l in range(MAX_LEVELS + 1):
         d.level_w[l] = 0.0
     if level_w is not None:

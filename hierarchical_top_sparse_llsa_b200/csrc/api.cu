@@ -47,6 +47,14 @@ inline int check_desc(const llsa_desc* d) {
 
 inline int n_level(const llsa_desc* d, int l) { return d->N >> (4 * l); }
 
+// Lc, the top level whose tokens are keys: coarse levels 2..Lc join the fine
+// keys (enrichment depth enrich_levels; 0 = all L levels, < 0 = none).
+inline int key_top(const llsa_desc* d) {
+  if (d->enrich_levels == 0) return d->L;
+  if (d->enrich_levels < 0) return 1;
+  return d->enrich_levels >= d->L - 1 ? d->L : 1 + d->enrich_levels;
+}
+
 inline float scale_of(const llsa_desc* d) {
   return d->sm_scale > 0.f ? d->sm_scale : 1.0f / sqrtf((float)d->D);
 }
@@ -69,9 +77,10 @@ inline WsLayout ws_layout(const llsa_desc* d) {
   };
   const size_t BH = (size_t)d->B * d->H;
   w.delta = take(BH * d->N * sizeof(float));
-  for (int l = 2; l <= d->L; ++l)
+  const int Lc = key_top(d);
+  for (int l = 2; l <= Lc; ++l)
     w.part[l] = take(BH * (size_t)(d->N >> 7) * d->topk * 2 * d->D * sizeof(float));
-  for (int l = 2; l <= d->L; ++l)
+  for (int l = 2; l <= Lc; ++l)
     w.coarse[l] = take(BH * (size_t)n_level(d, l) * 2 * d->D * sizeof(float));
   w.work = take(sizeof(int32_t));
   w.total = off;
@@ -89,7 +98,7 @@ inline TrWsLayout tr_ws_layout(const llsa_desc* d) {
   memset(&w, 0, sizeof(w));
   size_t off = 0;
   const size_t BH = (size_t)d->B * d->H;
-  for (int l = 1; l <= d->L; ++l) {
+  for (int l = 1; l <= key_top(d); ++l) {
     const int n = n_level(d, l);
     int nchunk = 0, rows = 0;
     transpose_chunking(n, &nchunk, &rows);
@@ -144,8 +153,9 @@ void fill_attn_common(AttnParams& p, const llsa_desc* d, const void* q, const vo
   p.q = q;
   p.k = k;
   p.v = v;
-  for (int l = 1; l <= d->L; ++l) p.idx[l] = idx->idx[l];
-  for (int l = 2; l <= d->L; ++l) {
+  const int Lc = key_top(d);
+  for (int l = 1; l <= Lc; ++l) p.idx[l] = idx->idx[l];
+  for (int l = 2; l <= Lc; ++l) {
     p.pk[l] = pyr->k[l];
     p.pv[l] = pyr->v[l];
     const float w = d->level_w[l] > 0.f ? d->level_w[l] : 1.0f;
@@ -155,19 +165,19 @@ void fill_attn_common(AttnParams& p, const llsa_desc* d, const void* q, const vo
   p.H = d->H;
   p.N = d->N;
   p.D = d->D;
-  p.L = d->L;
+  p.L = Lc;  // the kernels see only the levels whose tokens are keys
   p.K = d->topk;
   p.scale = scale_of(d);
 }
 
 bool coarse_kv_present(const llsa_desc* d, const llsa_pyramid* pyr) {
-  for (int l = 2; l <= d->L; ++l)
+  for (int l = 2; l <= key_top(d); ++l)
     if (pyr->k[l] == nullptr || pyr->v[l] == nullptr) return false;
   return true;
 }
 
-bool indices_present(const llsa_desc* d, const llsa_indices* idx) {
-  for (int l = 1; l <= d->L; ++l)
+bool indices_present(const llsa_desc* d, const llsa_indices* idx, int top) {
+  for (int l = 1; l <= top; ++l)
     if (idx->idx[l] == nullptr) return false;
   return true;
 }
@@ -237,7 +247,7 @@ int llsa_select(const llsa_desc* desc, const llsa_pyramid* pyr, const llsa_indic
                 void* stream) {
   int st = check_desc(desc);
   if (st != LLSA_OK) return st;
-  if (pyr == nullptr || out == nullptr || !indices_present(desc, out)) return LLSA_ERR_INVALID_ARG;
+  if (pyr == nullptr || out == nullptr || !indices_present(desc, out, desc->L)) return LLSA_ERR_INVALID_ARG;
   for (int l = 1; l <= desc->L; ++l)
     if (pyr->q[l] == nullptr || pyr->k[l] == nullptr) return LLSA_ERR_INVALID_ARG;
   const int BH = desc->B * desc->H;
@@ -263,7 +273,7 @@ int llsa_attn_fwd(const llsa_desc* desc, const void* q, const void* k, const voi
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || lse == nullptr ||
       idx == nullptr || pyr == nullptr)
     return LLSA_ERR_INVALID_ARG;
-  if (!indices_present(desc, idx) || !coarse_kv_present(desc, pyr)) return LLSA_ERR_INVALID_ARG;
+  if (!indices_present(desc, idx, key_top(desc)) || !coarse_kv_present(desc, pyr)) return LLSA_ERR_INVALID_ARG;
   AttnParams p;
   fill_attn_common(p, desc, q, k, v, pyr, idx);
   p.out = o;
@@ -296,7 +306,7 @@ int llsa_index_transpose(const llsa_desc* desc, const llsa_indices* idx, const l
                          void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
   int st = check_desc(desc);
   if (st != LLSA_OK) return st;
-  if (idx == nullptr || out == nullptr || ws == nullptr || !indices_present(desc, idx))
+  if (idx == nullptr || out == nullptr || ws == nullptr || !indices_present(desc, idx, key_top(desc)))
     return LLSA_ERR_INVALID_ARG;
   if (((uintptr_t)ws & 255) != 0) return LLSA_ERR_INVALID_ARG;
   const TrWsLayout w = tr_ws_layout(desc);
@@ -306,9 +316,9 @@ int llsa_index_transpose(const llsa_desc* desc, const llsa_indices* idx, const l
   p.BH = desc->B * desc->H;
   p.K = desc->topk;
   p.status = dev_status;
-  p.nlev = desc->L;
+  p.nlev = key_top(desc);
   int cta = 0, tile = 0, scan = 0;
-  for (int l = 1; l <= desc->L; ++l) {
+  for (int l = 1; l <= p.nlev; ++l) {
     if (out->row_ptr[l] == nullptr || out->col[l] == nullptr) return LLSA_ERR_INVALID_ARG;
     TransposeLevel& t = p.lv[l - 1];
     t.idx = idx->idx[l];
@@ -343,8 +353,9 @@ int llsa_attn_bwd(const llsa_desc* desc, const void* q, const void* k, const voi
       dk == nullptr || dv == nullptr || ws == nullptr)
     return LLSA_ERR_INVALID_ARG;
   if (((uintptr_t)ws & 255) != 0) return LLSA_ERR_INVALID_ARG;
-  if (!indices_present(desc, idx) || !coarse_kv_present(desc, pyr)) return LLSA_ERR_INVALID_ARG;
-  for (int l = 1; l <= desc->L; ++l)
+  const int p_top = key_top(desc);
+  if (!indices_present(desc, idx, p_top) || !coarse_kv_present(desc, pyr)) return LLSA_ERR_INVALID_ARG;
+  for (int l = 1; l <= p_top; ++l)
     if (csr->row_ptr[l] == nullptr || csr->col[l] == nullptr) return LLSA_ERR_INVALID_ARG;
   const WsLayout w = ws_layout(desc);
   if (ws_bytes < w.total) return LLSA_ERR_WORKSPACE;
@@ -353,13 +364,13 @@ int llsa_attn_bwd(const llsa_desc* desc, const void* q, const void* k, const voi
   p.o = o;
   p.lse_in = lse;
   p.dout = dout;
-  for (int l = 1; l <= desc->L; ++l) {
+  for (int l = 1; l <= p_top; ++l) {
     p.row_ptr[l] = csr->row_ptr[l];
     p.col[l] = csr->col[l];
   }
   char* base = static_cast<char*>(ws);
   p.delta = reinterpret_cast<float*>(base + w.delta);
-  for (int l = 2; l <= desc->L; ++l) {
+  for (int l = 2; l <= p_top; ++l) {
     p.part[l] = reinterpret_cast<float*>(base + w.part[l]);
     p.coarse[l] = reinterpret_cast<float*>(base + w.coarse[l]);
   }

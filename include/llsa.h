@@ -92,6 +92,13 @@ typedef struct {
    * Reweighting; the paper's setting is 16^l).  0 selects 1.  Entries 0, 1 and
    * above L are ignored. */
   float level_w[LLSA_MAX_LEVELS + 1];
+  /* Enrichment depth Le (Hierarchical KV Enrichment): the coarse levels whose
+   * pooled tokens join the keys are 2..Lc with Lc = min(L, 1 + Le).  0 selects
+   * all of them (Lc = L); a negative value selects none (Lc = 1: fine keys
+   * only).  Selection (llsa_select) always walks all L levels; the attention
+   * calls and llsa_index_transpose use levels 1..Lc only, and the I(l), CSR
+   * and pyramid entries of levels above Lc may be NULL there. */
+  int enrich_levels;
 } llsa_desc;
 
 /* fp32 pyramid, [B, H, N_l, D] per level; entry 0 is unused. */
@@ -148,14 +155,16 @@ LLSA_API int llsa_select(const llsa_desc* desc, const llsa_pyramid* pyr, const l
  * reweighting (Step 3; Building Blocks: Hierarchical KV Enrichment, KV
  * Reweighting).
  *   For query i of block b (i / 16 == b) the keys are the 16 fine tokens of
- *   every block in I(1)[b] (weight 1) and, for l = 2..L, the pooled tokens
+ *   every block in I(1)[b] (weight 1) and, for l = 2..Lc (Lc as enrich_levels
+ *   gives it; L by default), the pooled tokens
  *   K(l)[c], V(l)[c] for c in I(l)[b / 16^(l-1)] (weight level_w[l]):
  *     s_ij = sm_scale * q_i . k_j
  *     O_i  = sum_j w_j e^{s_ij} v_j / sum_j w_j e^{s_ij}
  *     lse_i = ln sum_j w_j e^{s_ij}          (natural log)
  *   A query without keys gets O_i = 0 and lse_i = -inf.
  *   idx may be any caller-made index lists (no hierarchy consistency needed).
- *   pyr: k[l], v[l] for l = 2..L.  o: [B, H, N, D] dtype.  lse: fp32 [B, H, N].
+ *   idx: I(1..Lc).  pyr: k[l], v[l] for l = 2..Lc.  o: [B, H, N, D] dtype.
+ *   lse: fp32 [B, H, N].
  *   dev_status: may be NULL.
  */
 LLSA_API int llsa_attn_fwd(const llsa_desc* desc, const void* q, const void* k, const void* v,
@@ -172,12 +181,12 @@ LLSA_API size_t llsa_transpose_workspace_bytes(const llsa_desc* desc);
 /*
  * llsa_index_transpose - sparse index transpose (Step 4; Building Blocks:
  * Sparse Index Transpose).
- *   For each level l = 1..L and (b, h): count the query tokens that kept each
+ *   For each level l = 1..Lc and (b, h): count the query tokens that kept each
  *   key token, prefix-sum the counts into row_ptr, and list the query tokens
  *   of each key in ascending order in col.  No dense mask is formed; the
  *   result is deterministic and uses no global atomics.
- *   idx: I(1..L), entries screened as the conventions above state.
- *   out: CSR of every level, written: row_ptr[l] int32 [B, H, N_l + 1],
+ *   idx: I(1..Lc), entries screened as the conventions above state.
+ *   out: CSR of levels 1..Lc, written: row_ptr[l] int32 [B, H, N_l + 1],
  *   col[l] int32 [B, H, N_l * K] (slots past row_ptr[N_l] set to -1).
  *   ws: device scratch of at least llsa_transpose_workspace_bytes(desc)
  *   bytes, 256-byte aligned, not read before it is written (a smaller or
@@ -207,7 +216,7 @@ LLSA_API size_t llsa_bwd_workspace_bytes(const llsa_desc* desc);
  *   o, lse: the outputs of llsa_attn_fwd (o must be valid but is not read:
  *   Delta_i = sum_j P_ij (dO_i . v_j) is recomputed from unrounded terms, as O
  *   itself is stored rounded to dtype).  dout: dO.  csr: llsa_index_transpose
- *   of the same idx.  dq, dk, dv: [B, H, N, D] dtype, written.
+ *   of the same idx (levels 1..Lc).  dq, dk, dv: [B, H, N, D] dtype, written.
  *   ws: device scratch of at least llsa_bwd_workspace_bytes(desc) bytes,
  *   256-byte aligned.  dev_status: may be NULL.
  */

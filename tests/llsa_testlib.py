@@ -59,14 +59,14 @@ def assert_close(got, want, dtype: str, what: str):
 
 
 def run_gpu(B, H, N, D, L, topk, dtype, inputs, level_w=None, ext_idx=None, bwd=True,
-            device="cuda", flags=0):
+            device="cuda", flags=0, enrich=0):
     """The whole path through the C ABI.  Returns numpy copies of everything."""
     import torch
 
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
     t = {k: torch.from_numpy(np.ascontiguousarray(v)).to(device=device, dtype=tdt) for k, v in inputs.items()}
     desc = llsa.make_desc(B, H, N, D, L, topk, llsa.BF16 if dtype == "bf16" else llsa.F32,
-                          level_w=level_w, flags=flags)
+                          level_w=level_w, flags=flags, enrich_levels=enrich)
     bufs = llsa.LlsaBuffers(desc, device, with_bwd=bwd)
     stream = torch.cuda.current_stream().cuda_stream
     st = bufs.status.data_ptr()
@@ -105,7 +105,7 @@ def run_gpu(B, H, N, D, L, topk, dtype, inputs, level_w=None, ext_idx=None, bwd=
     return out
 
 
-def run_oracle(inputs, L, topk, level_w=None, idx=None, bwd=True, pyr=None):
+def run_oracle(inputs, L, topk, level_w=None, idx=None, bwd=True, pyr=None, enrich=None):
     """The oracle on the same inputs.  ``idx`` replaces the selection;
     ``pyr`` (a dict with pq, pk, pv) replaces the pooling."""
     Q, K, V = inputs["q"], inputs["k"], inputs["v"]
@@ -114,12 +114,13 @@ def run_oracle(inputs, L, topk, level_w=None, idx=None, bwd=True, pyr=None):
     if pyr is None:
         pyr = {"pq": oracle.pool(Q, L), "pk": oracle.pool(K, L), "pv": oracle.pool(V, L)}
     sel = oracle.select_all(pyr["pq"], pyr["pk"], L, topk) if idx is None else idx
-    O, LSE = oracle.attn_fwd(Q, K, V, pyr["pk"], pyr["pv"], sel, L, scale, level_w)
+    O, LSE = oracle.attn_fwd(Q, K, V, pyr["pk"], pyr["pv"], sel, L, scale, level_w, enrich=enrich)
     res = {"pq": pyr["pq"], "pk": pyr["pk"], "pv": pyr["pv"], "idx": sel, "O": O, "LSE": LSE}
     if bwd:
         res["csr"] = {l: oracle.index_transpose(sel[l], Q.shape[2] // 16**l) for l in sel}
         res["dQ"], res["dK"], res["dV"] = oracle.attn_bwd(
-            Q, K, V, pyr["pk"], pyr["pv"], O, LSE, inputs["do"], sel, L, scale, level_w)
+            Q, K, V, pyr["pk"], pyr["pv"], O, LSE, inputs["do"], sel, L, scale, level_w,
+            enrich=enrich)
     return res
 
 

@@ -153,3 +153,26 @@ def test_reorder_argument_checks(lib, args, status):
     a.update(args)
     assert llsa.llsa_reorder(a["B"], a["H"], a["img_h"], a["img_w"], a["D"], a["dtype"], a["src"], a["dst"],
                              True, check=False) == status
+
+
+@pytest.mark.parametrize("enrich,top", [(0, 3), (1, 2), (2, 3), (5, 3), (-1, 1), (-4, 1)])
+def test_enrichment_depth_sizes_and_required_levels(lib, enrich, top):
+    # the attention-side workspaces cover levels 1..Lc only, Lc = min(L, 1 + depth)
+    B, H, N, D, L, K = 1, 2, 4096, 64, 3, 8
+    d = _desc(B=B, H=H, N=N, L=L)
+    d.enrich_levels = enrich
+    r256 = lambda x: (x + 255) // 256 * 256
+    want = r256(B * H * N * 4)
+    want += sum(r256(B * H * (N // 128) * K * 2 * D * 4) for _ in range(2, top + 1))
+    want += sum(r256(B * H * (N // 16**l) * 2 * D * 4) for l in range(2, top + 1))
+    want += 256
+    assert llsa.llsa_bwd_workspace_bytes(d) == want
+    assert llsa.llsa_transpose_workspace_bytes(d) == _transpose_ws_bytes(B, H, N, top)
+    # entries above Lc may be NULL: the workspace size check is what fails
+    ind, csr = llsa.LlsaIndices(), llsa.LlsaCsr()
+    for l in range(1, top + 1):
+        ind.idx[l] = csr.row_ptr[l] = csr.col[l] = 256
+    tw = llsa.llsa_transpose_workspace_bytes(d)
+    assert llsa.llsa_index_transpose(d, ind, csr, 256, tw - 1, check=False) == llsa.ERR_WORKSPACE
+    ind.idx[top] = 0  # a missing entry at or below Lc is an argument error
+    assert llsa.llsa_index_transpose(d, ind, csr, 256, tw, check=False) == llsa.ERR_INVALID_ARG

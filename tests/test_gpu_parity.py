@@ -239,3 +239,34 @@ def test_tcgen05_backward_external_indices_and_long_rows():
     r = run_oracle(x, L, K, idx=clean, level_w=lw)
     for name in ("dQ", "dK", "dV"):
         assert_close(g[name], r[name], "bf16", name)
+
+
+@pytest.mark.parametrize("enrich,flags", [
+    (-1, 0),
+    (1, 0),
+    (1, llsa.FLAG_FWD_TCGEN05 | llsa.FLAG_BWD_TCGEN05),
+    (2, 0),
+])
+def test_enrichment_depth(enrich, flags):
+    # L = 3 with the paper's level weights: depth 1 keeps the level-2 keys only,
+    # -1 the fine keys only, 2 every level (the default).  Selection walks all
+    # three levels either way; the key-major lists exist for levels 1..Lc.
+    B, H, N, D, L, K = 1, 3, 8192, 64, 3, 8
+    top = {-1: 1, 1: 2, 2: 3}[enrich]
+    x = _small(31, B, H, N, D)
+    lw = [0, 0] + [16.0**l for l in range(2, L + 1)]
+    g = run_gpu(B, H, N, D, L, K, "bf16", x, level_w=lw, flags=flags, enrich=enrich)
+    assert g["status"] == 0
+    r = run_oracle(x, L, K, level_w=lw, enrich=enrich)
+    for l in range(1, L + 1):
+        assert np.array_equal(g["idx"][l], r["idx"][l]), f"indices level {l}"
+    for l in range(1, top + 1):
+        rp, col = r["csr"][l]
+        assert np.array_equal(g["row_ptr"][l], rp), f"row_ptr level {l}"
+        assert np.array_equal(g["col"][l], col), f"col level {l}"
+    for name in ("O", "dQ", "dK", "dV"):
+        assert_close(g[name], r[name], "bf16", name)
+    assert_close(g["LSE"], r["LSE"], "bf16", "LSE")
+    if enrich != 2:  # the depth changes the result
+        full = run_oracle(x, L, K, level_w=lw, bwd=False)
+        assert not np.allclose(full["O"], r["O"], rtol=1e-3, atol=1e-3)
