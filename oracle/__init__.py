@@ -26,6 +26,10 @@ Parity status of each function (what pins it, in tests/test_oracle_*.py):
   attn_bwd         pinned: central finite differences of <dO, O>.
   zorder_index     pinned: the 4x4 grid written out by hand, a decoded
   reorder          token, 4x4-tile runs, round trips.
+  enriched_top     pinned: dense masked attention over levels 2..Lc,
+                   padded index lists, finite differences.
+  level_topk       pinned: flat exhaustive Top-K_1 under all-keeping upper
+                   levels, a planted descent that turns on K_2, padding.
 """
 
 from .llsa_oracle import (  # noqa: F401
@@ -35,6 +39,7 @@ from .llsa_oracle import (  # noqa: F401
     zorder_index,
     select_level,
     select_all,
+    level_topk,
     candidates_for_level,
     key_sets,
     attn_fwd,

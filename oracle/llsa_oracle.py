@@ -152,15 +152,26 @@ def select_level(
     return out
 
 
-def select_all(pyr_q: dict, pyr_k: dict, L: int, topk: int, factor: int = FACTOR) -> dict[int, np.ndarray]:
+def level_topk(topk, l: int) -> int:
+    """K_l, the number of keys kept at level l: topk itself when it is an
+    int, else topk[l] (a dict or a sequence indexed by level).  The pages fix
+    one K for every level; a K per level is the plainest reading of letting
+    K vary (Open Questions: adaptive K), with the same descent."""
+    return int(topk) if np.isscalar(topk) else int(topk[l])
+
+
+def select_all(pyr_q: dict, pyr_k: dict, L: int, topk, factor: int = FACTOR) -> dict[int, np.ndarray]:
     """Hierarchical Top-K from the coarsest level L down to level 1 (Step 2).
 
-    Returns {l: I(l)} for l = 1..L.
+    topk: one K for every level, or K_l per level (level_topk).  Level l then
+    keeps K_l of the factor * K_{l+1} children of its parent's kept keys.
+
+    Returns {l: I(l)} for l = 1..L, I(l) int32 [B, H, N_l, K_l].
     """
     idx = {}
     parent = None
     for l in range(L, 0, -1):
-        idx[l] = select_level(pyr_q[l], pyr_k[l], parent, topk, factor)
+        idx[l] = select_level(pyr_q[l], pyr_k[l], parent, level_topk(topk, l), factor)
         parent = idx[l]
     return idx
 
