@@ -52,6 +52,7 @@ class LlsaDesc(ctypes.Structure):
         ("L", ctypes.c_int), ("topk", ctypes.c_int), ("dtype", ctypes.c_int), ("flags", ctypes.c_int),
         ("sm_scale", ctypes.c_float), ("level_w", ctypes.c_float * (MAX_LEVELS + 1)),
         ("enrich_levels", ctypes.c_int),
+        ("topk_l", ctypes.c_int * (MAX_LEVELS + 1)),
     ]
 
 
@@ -120,11 +121,13 @@ def _check(status: int) -> int:
 
 
 def make_desc(B, H, N, D, L, topk, dtype, sm_scale=0.0, level_w=None, flags=0,
-              enrich_levels=0) -> LlsaDesc:
+              enrich_levels=0, topk_l=None) -> LlsaDesc:
     """Fill an llsa_desc; level_w is None (every weight 1) or indexable by level.
 
     enrich_levels is the enrichment depth: coarse levels 2..min(L, 1 + depth)
-    join the keys; 0 means all of them, a negative value none."""
+    join the keys; 0 means all of them, a negative value none.  topk_l is None
+    (topk at every level) or indexable by level: K_l, the keys kept at level l
+    (0 selects topk)."""
     d = LlsaDesc()
     d.B, d.H, d.N, d.D, d.L, d.topk = B, H, N, D, L, topk
     d.dtype = dtype
@@ -136,7 +139,17 @@ def make_desc(B, H, N, D, L, topk, dtype, sm_scale=0.0, level_w=None, flags=0,
     if level_w is not None:
         for l in range(2, L + 1):
             d.level_w[l] = float(level_w[l])
+    for l in range(MAX_LEVELS + 1):
+        d.topk_l[l] = 0
+    if topk_l is not None:
+        for l in range(1, L + 1):
+            d.topk_l[l] = int(topk_l[l])
     return d
+
+
+def level_topk(desc: LlsaDesc, l: int) -> int:
+    """K_l of a descriptor: the width of I(l)."""
+    return desc.topk_l[l] if desc.topk_l[l] > 0 else desc.topk
 
 
 # ------------------------------------------------------------ entry points
@@ -212,7 +225,7 @@ class LlsaBuffers:
         import torch
 
         self.desc = desc
-        B, H, N, D, L, K = desc.B, desc.H, desc.N, desc.D, desc.L, desc.topk
+        B, H, N, D, L = desc.B, desc.H, desc.N, desc.D, desc.L
         f32, i32 = torch.float32, torch.int32
         self.pq, self.pk, self.pv, self.idx, self.row_ptr, self.col = {}, {}, {}, {}, {}, {}
         self.pyramid = LlsaPyramid()
@@ -227,11 +240,12 @@ class LlsaBuffers:
             if l >= 2:
                 self.pv[l] = torch.empty(B, H, n, D, dtype=f32, device=device)
                 self.pyramid.v[l] = self.pv[l].data_ptr()
-            self.idx[l] = torch.empty(B, H, n, K, dtype=i32, device=device)
+            Kl = level_topk(desc, l)
+            self.idx[l] = torch.empty(B, H, n, Kl, dtype=i32, device=device)
             self.indices.idx[l] = self.idx[l].data_ptr()
             if with_bwd:
                 self.row_ptr[l] = torch.empty(B, H, n + 1, dtype=i32, device=device)
-                self.col[l] = torch.empty(B, H, n * K, dtype=i32, device=device)
+                self.col[l] = torch.empty(B, H, n * Kl, dtype=i32, device=device)
                 self.csr.row_ptr[l] = self.row_ptr[l].data_ptr()
                 self.csr.col[l] = self.col[l].data_ptr()
         self.ws_bytes = llsa_bwd_workspace_bytes(desc) if with_bwd else 0

@@ -27,6 +27,9 @@ constexpr bool kUseTcForward = false;
 // Likewise for the key-major backward pass; LLSA_FLAG_BWD_TCGEN05 selects it.
 constexpr bool kUseTcBackward = false;
 
+// K_l, the width of I(l): topk_l[l], or topk where that is 0.
+inline int k_level(const llsa_desc* d, int l) { return d->topk_l[l] > 0 ? d->topk_l[l] : d->topk; }
+
 inline int check_desc(const llsa_desc* d) {
   if (d == nullptr) return LLSA_ERR_INVALID_ARG;
   if (d->B < 1 || d->H < 1 || d->N < kBlock || d->D < 1 || d->L < 1 || d->topk < 1)
@@ -35,10 +38,15 @@ inline int check_desc(const llsa_desc* d) {
   if (d->dtype != LLSA_F32 && d->dtype != LLSA_BF16) return LLSA_ERR_INVALID_ARG;
   if (d->D != 64 && d->D != 128) return LLSA_ERR_UNSUPPORTED;
   if (d->L > kMaxL || d->topk > kMaxK) return LLSA_ERR_UNSUPPORTED;
+  for (int l = 1; l <= d->L; ++l) {
+    if (d->topk_l[l] < 0) return LLSA_ERR_INVALID_ARG;
+    if (d->topk_l[l] > kMaxK) return LLSA_ERR_UNSUPPORTED;
+  }
   const long long span = 1LL << (4 * d->L);
   if (d->N % span != 0) return LLSA_ERR_INVALID_ARG;
   if ((long long)d->B * d->H > 65535) return LLSA_ERR_UNSUPPORTED;  // grid.y
-  if ((long long)(d->N / kBlock) * d->topk > 0x7fffffffLL) return LLSA_ERR_UNSUPPORTED;
+  for (int l = 1; l <= d->L; ++l)  // CSR offsets are int32
+    if ((long long)(d->N >> (4 * l)) * k_level(d, l) > 0x7fffffffLL) return LLSA_ERR_UNSUPPORTED;
   if (!(d->sm_scale >= 0.f) || isinf(d->sm_scale)) return LLSA_ERR_INVALID_ARG;
   for (int l = 2; l <= d->L; ++l)
     if (!(d->level_w[l] >= 0.f) || isinf(d->level_w[l])) return LLSA_ERR_INVALID_ARG;
@@ -46,6 +54,7 @@ inline int check_desc(const llsa_desc* d) {
 }
 
 inline int n_level(const llsa_desc* d, int l) { return d->N >> (4 * l); }
+
 
 // Lc, the top level whose tokens are keys: coarse levels 2..Lc join the fine
 // keys (enrichment depth enrich_levels; 0 = all L levels, < 0 = none).
@@ -79,7 +88,7 @@ inline WsLayout ws_layout(const llsa_desc* d) {
   w.delta = take(BH * d->N * sizeof(float));
   const int Lc = key_top(d);
   for (int l = 2; l <= Lc; ++l)
-    w.part[l] = take(BH * (size_t)(d->N >> 7) * d->topk * 2 * d->D * sizeof(float));
+    w.part[l] = take(BH * (size_t)(d->N >> 7) * k_level(d, l) * 2 * d->D * sizeof(float));
   for (int l = 2; l <= Lc; ++l)
     w.coarse[l] = take(BH * (size_t)n_level(d, l) * 2 * d->D * sizeof(float));
   w.work = take(sizeof(int32_t));
@@ -166,7 +175,12 @@ void fill_attn_common(AttnParams& p, const llsa_desc* d, const void* q, const vo
   p.N = d->N;
   p.D = d->D;
   p.L = Lc;  // the kernels see only the levels whose tokens are keys
-  p.K = d->topk;
+  p.K = k_level(d, 1);
+  p.Kc = 0;
+  for (int l = 1; l <= Lc; ++l) {
+    p.Kl[l] = k_level(d, l);
+    if (l >= 2) p.Kc += p.Kl[l];
+  }
   p.scale = scale_of(d);
 }
 
@@ -258,7 +272,8 @@ int llsa_select(const llsa_desc* desc, const llsa_pyramid* pyr, const llsa_indic
     p.parent = (l == desc->L) ? nullptr : out->idx[l + 1];
     p.out = out->idx[l];
     p.n = n_level(desc, l);
-    p.K = desc->topk;
+    p.K = k_level(desc, l);
+    p.Kp = (l == desc->L) ? 0 : k_level(desc, l + 1);
     st = launch_status(launch_select_level(p, BH, desc->D, (cudaStream_t)stream));
     if (st != LLSA_OK) return st;
   }
@@ -314,7 +329,6 @@ int llsa_index_transpose(const llsa_desc* desc, const llsa_indices* idx, const l
   TransposeParams p;
   memset(&p, 0, sizeof(p));
   p.BH = desc->B * desc->H;
-  p.K = desc->topk;
   p.status = dev_status;
   p.nlev = key_top(desc);
   int cta = 0, tile = 0, scan = 0;
@@ -326,6 +340,7 @@ int llsa_index_transpose(const llsa_desc* desc, const llsa_indices* idx, const l
     t.col = out->col[l];
     t.cnt = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + w.off[l]);
     t.n = n_level(desc, l);
+    t.K = k_level(desc, l);
     transpose_chunking(t.n, &t.nchunk, &t.rows);
     t.cta_begin = cta;
     t.tile_begin = tile;

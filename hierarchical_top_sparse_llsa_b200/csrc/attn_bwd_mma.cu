@@ -144,8 +144,9 @@ bwd_q_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
     for (int l = 2; l <= p.L; ++l) {
       const int nl = p.N >> (4 * l);
       const int a = b0 >> (4 * (l - 1));
-      const int c = (lane < K) ? p.idx[l][((size_t)bh * nl + a) * K + lane] : -1;
-      const bool u = warp_row_used(c, lane, nl, lane < K, flags);
+      const int Kl = p.Kl[l];
+      const int c = (lane < Kl) ? p.idx[l][((size_t)bh * nl + a) * Kl + lane] : -1;
+      const bool u = warp_row_used(c, lane, nl, lane < Kl, flags);
       const unsigned m = __ballot_sync(0xffffffffu, u);
       if (u) {
         const int pos = n + __popc(m & ((1u << lane) - 1u));
@@ -411,7 +412,7 @@ bwd_q_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
         const int ck_idx = ct * 16 + g + 8 * half;
         if (ck_idx < nc) {
           const int l = clist[ck_idx] >> 24;
-          float* part = p.part[l] + ((((size_t)bh * NG + grp) * K + cslot[ck_idx]) * 2 + kv) * D;
+          float* part = p.part[l] + ((((size_t)bh * NG + grp) * p.Kl[l] + cslot[ck_idx]) * 2 + kv) * D;
 #pragma unroll
           for (int j = 0; j < NTW; ++j)
             *reinterpret_cast<float2*>(part + 8 * (j0 + j) + 2 * t) =
@@ -683,7 +684,7 @@ cudaError_t launch_typed(const AttnParams& p, const CUtensorMap* maps, cudaStrea
   constexpr int TILE = 32 * D;
   const int BH = p.B * p.H;
   const int n1 = p.N / kBlock;
-  const int nct = ((p.L - 1) * p.K + 15) / 16;
+  const int nct = (p.Kc + 15) / 16;
   // pass 1
   const size_t smem1 = 1024 + (size_t)kQWarps * TILE * (2 + 2 * kRing) + 2 * (size_t)nct * TILE +
                        nct * 16 * sizeof(float) + kQWarps * (1 + kRing) * 8 + 2 * nct * 16 * sizeof(int);

@@ -76,8 +76,8 @@ bwd_query_simt_kernel(AttnParams p, int G) {
 
   // zero this CTA's partial slots (levels 2..L)
   for (int l = 2; l <= p.L; ++l) {
-    float* part = p.part[l] + ((size_t)bh * NG + g) * K * 2 * D;
-    for (int e = tid; e < K * 2 * D; e += 256) part[e] = 0.f;
+    float* part = p.part[l] + ((size_t)bh * NG + g) * p.Kl[l] * 2 * D;
+    for (int e = tid; e < p.Kl[l] * 2 * D; e += 256) part[e] = 0.f;
   }
   int flags = 0;
   for (int bb = 0; bb < G; ++bb) {
@@ -178,7 +178,7 @@ bwd_query_simt_kernel(AttnParams p, int G) {
           gk = fmaf(dss[r][j], qs[r][d], gk);
           gv = fmaf(ps[r][j], dos[r][d], gv);
         }
-        float* part = p.part[lv] + (((size_t)bh * NG + g) * K + kl.slot[t0 + j]) * 2 * D;
+        float* part = p.part[lv] + (((size_t)bh * NG + g) * p.Kl[lv] + kl.slot[t0 + j]) * 2 * D;
         part[d] += gk * p.scale;
         part[D + d] += gv;
       }
@@ -198,7 +198,7 @@ __global__ void bwd_coarse_reduce_kernel(AttnParams p, int l) {
   __shared__ int s_q[kReduceChunk], s_slot[kReduceChunk];
   const int c = blockIdx.x;
   const int bh = blockIdx.y;
-  const int D = p.D, K = p.K;
+  const int D = p.D, K = p.Kl[l];
   const int nl = p.N >> (4 * l);
   const int NG = p.N >> 7;
   const int span = 2 << (4 * (l - 2));  // groups of 8 query blocks under a level-l token
@@ -362,7 +362,7 @@ cudaError_t launch_typed(const AttnParams& p, cudaStream_t s) {
 // group (thread per (token, slot, kv, d); the groups in ascending order), so
 // the key-major gather reads one group per entry.
 __global__ void bwd_span_reduce_kernel(AttnParams p, int l) {
-  const int D = p.D, K = p.K;
+  const int D = p.D, K = p.Kl[l];
   const int nl = p.N >> (4 * l);
   const int NG = p.N >> 7;
   const int span = 2 << (4 * (l - 2));
@@ -383,7 +383,7 @@ __global__ void bwd_span_reduce_kernel(AttnParams p, int l) {
 cudaError_t launch_coarse_reduce(const AttnParams& p, cudaStream_t s) {
   for (int l = 2; l <= p.L; ++l) {
     if (l >= 3) {
-      const size_t total = (size_t)p.B * p.H * (p.N >> (4 * l)) * p.K * 2 * p.D;
+      const size_t total = (size_t)p.B * p.H * (p.N >> (4 * l)) * p.Kl[l] * 2 * p.D;
       int blocks = (int)((total + 255) / 256);
       if (blocks > 148 * 16) blocks = 148 * 16;
       bwd_span_reduce_kernel<<<blocks, 256, 0, s>>>(p, l);

@@ -192,8 +192,9 @@ attn_fwd_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
     for (int l = 2; l <= p.L; ++l) {
       const int nl = p.N >> (4 * l);
       const int a = b0 >> (4 * (l - 1));
-      const int c = (lane < K) ? p.idx[l][((size_t)bh * nl + a) * K + lane] : -1;
-      const bool u = warp_row_used(c, lane, nl, lane < K, flags);
+      const int Kl = p.Kl[l];
+      const int c = (lane < Kl) ? p.idx[l][((size_t)bh * nl + a) * Kl + lane] : -1;
+      const bool u = warp_row_used(c, lane, nl, lane < Kl, flags);
       const unsigned m = __ballot_sync(0xffffffffu, u);
       if (u) clist[n + __popc(m & ((1u << lane) - 1u))] = (l << 24) | c;
       n += __popc(m);
@@ -355,7 +356,7 @@ attn_fwd_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
 template <int D>
 cudaError_t launch_typed(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s) {
   constexpr int TILE = 32 * D;
-  const int nct = ((p.L - 1) * p.K + 15) / 16;
+  const int nct = (p.Kc + 15) / 16;
   const size_t smem = 1024 + (size_t)kFwdWarps * TILE * (2 + 2 * kStages) + 2 * (size_t)nct * TILE +
                       nct * 16 * sizeof(float) + kFwdWarps * (2 + kStages) * 8 + nct * 16 * sizeof(int);
   cudaError_t e = cudaFuncSetAttribute(attn_fwd_mma_kernel<D>,

@@ -45,8 +45,9 @@ __device__ __forceinline__ int build_key_list(KeyList& kl, const AttnParams& p, 
   for (int l = 2; l <= p.L; ++l) {
     const int nl = p.N >> (4 * l);
     const int a = b >> (4 * (l - 1));
-    const int c = (lane < K) ? p.idx[l][((size_t)bh * nl + a) * K + lane] : -1;
-    const bool u = warp_row_used(c, lane, nl, lane < K, flags);
+    const int Kl = p.Kl[l];
+    const int c = (lane < Kl) ? p.idx[l][((size_t)bh * nl + a) * Kl + lane] : -1;
+    const bool u = warp_row_used(c, lane, nl, lane < Kl, flags);
     const unsigned m = __ballot_sync(0xffffffffu, u);
     if (u) {
       const int pos = n + __popc(m & ((1u << lane) - 1u));

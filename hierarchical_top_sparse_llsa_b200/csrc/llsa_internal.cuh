@@ -123,10 +123,11 @@ struct PoolParams {
 struct SelectParams {
   const float* ql;       // Q(l) [BH, n, D]
   const float* kl;       // K(l) [BH, n, D]
-  const int32_t* parent; // I(l+1) [BH, n/16, K] or nullptr at level L
+  const int32_t* parent; // I(l+1) [BH, n/16, Kp] or nullptr at level L
   int32_t* out;          // I(l) [BH, n, K]
   int n;                 // N_l
-  int K;
+  int K;                 // K_l, kept keys per row at this level
+  int Kp;                // K_{l+1}, the parent row's width
 };
 
 struct TransposeLevel {
@@ -135,6 +136,7 @@ struct TransposeLevel {
   int32_t* col;
   int32_t* cnt;    // workspace [BH][nchunk][n]: per-chunk key counts, then cursors
   int n;           // N_l (queries == keys at level l)
+  int K;           // K_l, the width of an index row
   int nchunk;      // row chunks per (b, h)
   int rows;        // rows per chunk
   int cta_begin;   // first CTA of this level in the count and fill grids
@@ -145,7 +147,7 @@ struct TransposeLevel {
 struct TransposeParams {
   TransposeLevel lv[kMaxL];
   int nlev;
-  int BH, K;
+  int BH;
   int32_t* status;
 };
 
@@ -168,11 +170,13 @@ struct AttnParams {
   void* dk;
   void* dv;
   float* delta;                 // [BH, N]
-  float* part[kMaxL + 1];       // [BH, N/128, K, 2, D] per coarse level (groups of 8 query blocks)
+  float* part[kMaxL + 1];       // [BH, N/128, K_l, 2, D] per coarse level (groups of 8 query blocks)
   float* coarse[kMaxL + 1];     // [BH, N_l, 2, D] per coarse level
   int32_t* work;                // pass-3 work counter (zeroed by pass 1)
   int32_t* status;
-  int B, H, N, D, L, K;
+  int B, H, N, D, L, K;  // L: top key level (Lc); K = K_1, the fine blocks per query block
+  int Kl[kMaxL + 1];      // K_l, the width of I(l) (Kl[1] == K)
+  int Kc;                 // coarse keys per query block at most: sum of K_l, l = 2..L
   float scale;
 };
 

@@ -94,8 +94,9 @@ select_kernel(SelectParams p) {
     if (!top) {
       const int np = n / kBlock;
       int f = 0;
-      const int c = (lane < K) ? p.parent[((size_t)bh * np + grp) * K + lane] : -1;
-      const bool u = warp_row_used(c, lane, np, lane < K, f);
+      const int Kp = p.Kp;  // the parent row's width
+      const int c = (lane < Kp) ? p.parent[((size_t)bh * np + grp) * Kp + lane] : -1;
+      const bool u = warp_row_used(c, lane, np, lane < Kp, f);
       const unsigned msk = __ballot_sync(0xffffffffu, u);
       if (u) parents[__popc(msk & ((1u << lane) - 1u))] = c;
       m = __popc(msk);

@@ -69,7 +69,7 @@ tr_count_kernel(TransposeParams p) {
   const TransposeLevel L = p.lv[level_of(p, blockIdx.x, kChunkGrid)];
   const int local = blockIdx.x - L.cta_begin;
   const int bh = local / L.nchunk, ch = local % L.nchunk;
-  const int n = L.n, K = p.K;
+  const int n = L.n, K = L.K;
   const int r0 = ch * L.rows, r1 = min(n, r0 + L.rows);
   const int32_t* I = L.idx + (size_t)bh * n * K;
   int32_t* cnt = L.cnt + ((size_t)bh * L.nchunk + ch) * n;
@@ -158,7 +158,7 @@ tr_scan_kernel(TransposeParams p) {
   __shared__ int warp_tot[kScanThreads / 32];
   const TransposeLevel L = p.lv[level_of(p, blockIdx.x, kScanGrid)];
   const int bh = blockIdx.x - L.scan_begin;
-  const int n = L.n, K = p.K;
+  const int n = L.n, K = L.K;
   int32_t* row_ptr = L.row_ptr + (size_t)bh * (n + 1);
   int32_t* col = L.col + (size_t)bh * n * K;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -203,7 +203,7 @@ tr_fill_kernel(TransposeParams p) {
   const TransposeLevel L = p.lv[level_of(p, blockIdx.x, kChunkGrid)];
   const int local = blockIdx.x - L.cta_begin;
   const int bh = local / L.nchunk, ch = local % L.nchunk;
-  const int n = L.n, K = p.K;
+  const int n = L.n, K = L.K;
   const int r0 = ch * L.rows, r1 = min(n, r0 + L.rows);
   const int32_t* I = L.idx + (size_t)bh * n * K;
   const int32_t* start = L.cnt + ((size_t)bh * L.nchunk + ch) * n;

@@ -14,7 +14,8 @@
  *    token is a 16-token query/key block.  N must be a multiple of 16^L.
  *  - Layout: every tensor is contiguous [B, H, tokens, D], D innermost.
  *    Q, K, V, O, dO, dQ, dK, dV hold `dtype` elements; pyramids are fp32.
- *  - Index lists I(l): int32 [B, H, N_l, topk].  Row q lists the level-l key
+ *  - Index lists I(l): int32 [B, H, N_l, K_l] (K_l = topk_l[l], else topk).
+ *    Row q lists the level-l key
  *    tokens kept for level-l query token q, ascending, padded with -1 at the
  *    tail.  Kernels that read index lists use an entry iff it lies in
  *    [0, N_l) and is larger than every entry used before it in the row; any
@@ -56,7 +57,7 @@ enum { LLSA_F32 = 0, LLSA_BF16 = 1 };
 enum {
   LLSA_OK = 0,
   LLSA_ERR_INVALID_ARG = 1, /* NULL pointer, bad shape, N not a multiple of 16^L, ... */
-  LLSA_ERR_UNSUPPORTED = 2, /* D not in {64, 128}, topk > 32, L > 6, ... */
+  LLSA_ERR_UNSUPPORTED = 2, /* D not in {64, 128}, topk or a K_l > 32, L > 6, ... */
   LLSA_ERR_LAUNCH = 3,      /* a kernel launch failed (cudaGetLastError) */
   LLSA_ERR_WORKSPACE = 4    /* workspace smaller than the matching *_workspace_bytes() */
 };
@@ -84,7 +85,7 @@ enum {
 typedef struct {
   int B, H, N, D; /* batch, heads, fine tokens, head dim (64 or 128) */
   int L;          /* number of pooled levels, 1 <= L <= LLSA_MAX_LEVELS */
-  int topk;       /* K, kept keys per level, 1 <= K <= LLSA_MAX_TOPK */
+  int topk;       /* K, kept keys per level, 1 <= K <= LLSA_MAX_TOPK (see topk_l) */
   int dtype;      /* LLSA_F32 or LLSA_BF16 */
   int flags;      /* LLSA_FLAG_* bits; other bits must be 0 */
   float sm_scale; /* softmax scale; 0 selects 1/sqrt(D) */
@@ -99,6 +100,11 @@ typedef struct {
    * calls and llsa_index_transpose use levels 1..Lc only, and the I(l), CSR
    * and pyramid entries of levels above Lc may be NULL there. */
   int enrich_levels;
+  /* topk_l[l], l = 1..L: K_l, the keys kept at level l (a Top-K per level;
+   * level l keeps K_l of the 16 * K_{l+1} children of its parent's keys).
+   * 0 selects topk; entries 0 and above L are ignored.  I(l) rows and the
+   * level-l CSR then have width K_l. */
+  int topk_l[LLSA_MAX_LEVELS + 1];
 } llsa_desc;
 
 /* fp32 pyramid, [B, H, N_l, D] per level; entry 0 is unused. */
@@ -108,13 +114,13 @@ typedef struct {
   float* v[LLSA_MAX_LEVELS + 1]; /* levels 2..L (level-1 pooled V is never a key) */
 } llsa_pyramid;
 
-/* I(l), int32 [B, H, N_l, topk] for l = 1..L; entry 0 is unused. */
+/* I(l), int32 [B, H, N_l, K_l] for l = 1..L; entry 0 is unused. */
 typedef struct {
   int32_t* idx[LLSA_MAX_LEVELS + 1];
 } llsa_indices;
 
 /* Key-major lists per level l = 1..L: row_ptr int32 [B, H, N_l + 1] and
- * col int32 [B, H, N_l * topk].  Row c of (b, h) is
+ * col int32 [B, H, N_l * K_l].  Row c of (b, h) is
  * col[row_ptr[c] .. row_ptr[c+1]), the level-l query tokens that kept key c,
  * ascending; offsets restart at 0 for every (b, h); col past row_ptr[N_l] is -1. */
 typedef struct {
@@ -142,7 +148,7 @@ LLSA_API int llsa_pool(const llsa_desc* desc, const void* q, const void* k, cons
  *   Level l < L: query token q scores only the 16 children of each key kept
  *   by its parent q/16 in I(l+1).  Score = Q(l)[q] . K(l)[c], unscaled, in
  *   fp32 summed over d = 0..D-1 left to right with one rounding per multiply
- *   and per add (no FMA).  The min(K, #candidates) best scores are kept;
+ *   and per add (no FMA).  The min(K_l, #candidates) best scores are kept;
  *   equal scores (IEEE ==) go to the lower key index.  Rows are stored
  *   ascending with -1 padding.
  *   pyr: q[l], k[l] for l = 1..L (from llsa_pool).  out: I(1..L), written.

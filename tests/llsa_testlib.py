@@ -59,14 +59,14 @@ def assert_close(got, want, dtype: str, what: str):
 
 
 def run_gpu(B, H, N, D, L, topk, dtype, inputs, level_w=None, ext_idx=None, bwd=True,
-            device="cuda", flags=0, enrich=0):
+            device="cuda", flags=0, enrich=0, topk_l=None):
     """The whole path through the C ABI.  Returns numpy copies of everything."""
     import torch
 
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
     t = {k: torch.from_numpy(np.ascontiguousarray(v)).to(device=device, dtype=tdt) for k, v in inputs.items()}
     desc = llsa.make_desc(B, H, N, D, L, topk, llsa.BF16 if dtype == "bf16" else llsa.F32,
-                          level_w=level_w, flags=flags, enrich_levels=enrich)
+                          level_w=level_w, flags=flags, enrich_levels=enrich, topk_l=topk_l)
     bufs = llsa.LlsaBuffers(desc, device, with_bwd=bwd)
     stream = torch.cuda.current_stream().cuda_stream
     st = bufs.status.data_ptr()

@@ -176,3 +176,26 @@ def test_enrichment_depth_sizes_and_required_levels(lib, enrich, top):
     assert llsa.llsa_index_transpose(d, ind, csr, 256, tw - 1, check=False) == llsa.ERR_WORKSPACE
     ind.idx[top] = 0  # a missing entry at or below Lc is an argument error
     assert llsa.llsa_index_transpose(d, ind, csr, 256, tw, check=False) == llsa.ERR_INVALID_ARG
+
+
+def test_topk_per_level_sizes_and_checks(lib):
+    B, H, N, D, L = 1, 2, 4096, 64, 3
+    kl = {1: 12, 2: 4, 3: 2}
+    d = llsa.make_desc(B, H, N, D, L, 8, llsa.BF16, topk_l=[0, 12, 4, 2])
+    r256 = lambda x: (x + 255) // 256 * 256
+    want = r256(B * H * N * 4)
+    want += sum(r256(B * H * (N // 128) * kl[l] * 2 * D * 4) for l in range(2, L + 1))
+    want += sum(r256(B * H * (N // 16**l) * 2 * D * 4) for l in range(2, L + 1))
+    want += 256
+    assert llsa.llsa_bwd_workspace_bytes(d) == want
+    assert llsa.level_topk(d, 1) == 12 and llsa.level_topk(d, 3) == 2
+    d0 = llsa.make_desc(B, H, N, D, L, 8, llsa.BF16, topk_l=[0, 0, 5, 0])
+    assert [llsa.level_topk(d0, l) for l in (1, 2, 3)] == [8, 5, 8]
+    bad = llsa.make_desc(B, H, N, D, L, 8, llsa.BF16, topk_l=[0, 33, 0, 0])
+    assert llsa.llsa_bwd_workspace_bytes(bad) == 0
+    bad = llsa.make_desc(B, H, N, D, L, 8, llsa.BF16, topk_l=[0, 0, -1, 0])
+    assert llsa.llsa_bwd_workspace_bytes(bad) == 0
+    pyr, ind = llsa.LlsaPyramid(), llsa.LlsaIndices()
+    assert llsa.llsa_select(bad, pyr, ind, check=False) == llsa.ERR_INVALID_ARG
+    bad.topk_l[2] = 40
+    assert llsa.llsa_select(bad, pyr, ind, check=False) == llsa.ERR_UNSUPPORTED

@@ -270,3 +270,28 @@ def test_enrichment_depth(enrich, flags):
     if enrich != 2:  # the depth changes the result
         full = run_oracle(x, L, K, level_w=lw, bwd=False)
         assert not np.allclose(full["O"], r["O"], rtol=1e-3, atol=1e-3)
+
+
+@pytest.mark.parametrize("dtype,flags,kl", [
+    ("bf16", 0, {1: 12, 2: 4, 3: 2}),
+    ("bf16", 0, {1: 4, 2: 16, 3: 1}),
+    ("bf16", 0, {1: 20, 2: 1, 3: 1}),   # 16 level-1 candidates: four pads per row
+    ("bf16", llsa.FLAG_FWD_TCGEN05 | llsa.FLAG_BWD_TCGEN05, {1: 12, 2: 4, 3: 2}),
+    ("f32", 0, {1: 6, 2: 3, 3: 2}),
+])
+def test_topk_per_level(dtype, flags, kl):
+    # K_l kept keys at level l: I(l) rows of width K_l, level l choosing among
+    # the 16 * K_{l+1} children of its parent's keys; the paper weights make
+    # the coarse keys count.
+    B, H, N, D, L = 1, 3, 8192, 64, 3
+    x = _small(32, B, H, N, D, dtype)
+    lw = [0, 0] + [16.0**l for l in range(2, L + 1)]
+    g = run_gpu(B, H, N, D, L, 8, dtype, x, level_w=lw, flags=flags, topk_l=[0] + [kl[l] for l in (1, 2, 3)])
+    assert g["status"] == 0
+    r = run_oracle(x, L, kl, level_w=lw)
+    w = workloads.Workload("kl", B, H, N, D, dtype, L, 8, 0)
+    for l in range(1, L + 1):
+        assert g["idx"][l].shape[-1] == kl[l]
+    _compare(w, g, r, slice(None), True)
+    if kl[1] > 16 * kl[2]:
+        assert np.all((g["idx"][1] >= 0).sum(-1) == 16 * kl[2])
