@@ -409,17 +409,26 @@ def run_ours(args, rank, world, local_rank):
     sh = stream.cuda_stream
     st = bufs.status.data_ptr()
 
+    fuse = args.fuse_select
+
     def step(tin, ev=None, sh=sh):
+        # ev given: the stages as separate calls with events between them;
+        # otherwise the step as timed (with --fuse-select, the level-1
+        # selection inside the forward)
         q, k, v = tin["q"].data_ptr(), tin["k"].data_ptr(), tin["v"].data_ptr()
         if ev is not None:
             ev[0].record(stream)
         llsa.llsa_pool(desc, q, k, v, bufs.pyramid, sh)
         if ev is not None:
             ev[1].record(stream)
-        llsa.llsa_select(desc, bufs.pyramid, bufs.indices, sh)
-        if ev is not None:
-            ev[2].record(stream)
-        llsa.llsa_attn_fwd(desc, q, k, v, bufs.pyramid, bufs.indices, o.data_ptr(), lse.data_ptr(), st, sh)
+        if fuse and ev is None:
+            llsa.llsa_select_attn_fwd(desc, q, k, v, bufs.pyramid, bufs.indices, o.data_ptr(), lse.data_ptr(),
+                                      st, sh)
+        else:
+            llsa.llsa_select(desc, bufs.pyramid, bufs.indices, sh)
+            if ev is not None:
+                ev[2].record(stream)
+            llsa.llsa_attn_fwd(desc, q, k, v, bufs.pyramid, bufs.indices, o.data_ptr(), lse.data_ptr(), st, sh)
         if ev is not None:
             ev[3].record(stream)
         if w.backward:
@@ -476,17 +485,16 @@ def run_ours(args, rank, world, local_rank):
         if graph is not None:
             graph.replay()
         else:
-            step(t_in, evs[s])
+            step(t_in)
     t_end.record(stream)
     torch.cuda.synchronize()
     barrier()
     if sampler:
         sampler.__exit__()
     ms = t_start.elapsed_time(t_end) / args.steps
-    if graph is not None:  # stage breakdown from direct calls
-        for s in range(args.steps):
-            step(t_in, evs[s])
-        torch.cuda.synchronize()
+    for s in range(args.steps):  # stage breakdown from separate direct calls
+        step(t_in, evs[s])
+    torch.cuda.synchronize()
     stage_ms = {}
     names = STAGES if w.backward else STAGES[:3]
     for i, name in enumerate(names):
@@ -568,7 +576,9 @@ def run_ours(args, rank, world, local_rank):
     attn_ms = stage_ms["fwd"] + stage_ms.get("bwd", 0.0)
     attn_flops = work["fwd"]["flops"] + (work["bwd"]["flops"] if w.backward else 0)
     sel_ms = stage_ms["pool"] + stage_ms["select"]
-    nlaunch = sum(launches_per_step(w.L)[n] for n in names)
+    # the fused call saves the level-1 selection launch on the bf16 warp-MMA forward
+    fused_saves = fuse and w.dtype == "bf16" and not args.fwd_tcgen05
+    nlaunch = sum(launches_per_step(w.L)[n] for n in names) - (1 if fused_saves else 0)
     line = {
         "metric": METRIC, "value": world * tokens / (ms * 1e-3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
@@ -586,6 +596,7 @@ def run_ours(args, rank, world, local_rank):
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
         "gpu_launches": nlaunch * args.steps,
         "cuda_graph": graph_note,
+        "select_in_fwd": fuse,
         "clocks": sampler.summary() if sampler else None,
     }
     print(json.dumps(line), flush=True)
@@ -609,6 +620,9 @@ def main():
                     help="run the key-major backward pass on the tcgen05 kernel (bf16, D=64)")
     ap.add_argument("--fwd-tcgen05", action="store_true",
                     help="run the forward on the tcgen05 kernel (bf16, D=64)")
+    ap.add_argument("--fuse-select", action="store_true",
+                    help="time llsa_select_attn_fwd (level-1 selection in the forward's prologue) "
+                         "instead of llsa_select + llsa_attn_fwd")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         ap.error("--warmup must be at least 3")

@@ -35,6 +35,7 @@ EXPORTED = (
     "llsa_pool",
     "llsa_select",
     "llsa_attn_fwd",
+    "llsa_select_attn_fwd",
     "llsa_transpose_workspace_bytes",
     "llsa_index_transpose",
     "llsa_bwd_workspace_bytes",
@@ -92,6 +93,8 @@ def lib() -> ctypes.CDLL:
             "llsa_select": (ctypes.c_int, [P(LlsaDesc), P(LlsaPyramid), P(LlsaIndices), vp]),
             "llsa_attn_fwd": (ctypes.c_int, [P(LlsaDesc), vp, vp, vp, P(LlsaPyramid), P(LlsaIndices),
                                              vp, vp, vp, vp]),
+            "llsa_select_attn_fwd": (ctypes.c_int, [P(LlsaDesc), vp, vp, vp, P(LlsaPyramid), P(LlsaIndices),
+                                                    vp, vp, vp, vp]),
             "llsa_transpose_workspace_bytes": (ctypes.c_size_t, [P(LlsaDesc)]),
             "llsa_index_transpose": (ctypes.c_int, [P(LlsaDesc), P(LlsaIndices), P(LlsaCsr), vp,
                                                     ctypes.c_size_t, vp, vp]),
@@ -166,6 +169,12 @@ def llsa_select(desc, pyramid, indices, stream=0, check=True):
 def llsa_attn_fwd(desc, q, k, v, pyramid, indices, o, lse, dev_status=None, stream=0, check=True):
     st = lib().llsa_attn_fwd(ctypes.byref(desc), q, k, v, ctypes.byref(pyramid), ctypes.byref(indices),
                              o, lse, dev_status, stream)
+    return _check(st) if check else st
+
+
+def llsa_select_attn_fwd(desc, q, k, v, pyramid, indices, o, lse, dev_status=None, stream=0, check=True):
+    st = lib().llsa_select_attn_fwd(ctypes.byref(desc), q, k, v, ctypes.byref(pyramid),
+                                    ctypes.byref(indices), o, lse, dev_status, stream)
     return _check(st) if check else st
 
 

@@ -13,6 +13,8 @@ namespace llsa {
 cudaError_t launch_attn_fwd_simt(const AttnParams& p, int dtype, cudaStream_t s);
 cudaError_t launch_attn_bwd_simt(const AttnParams& p, int dtype, cudaStream_t s);
 cudaError_t launch_attn_fwd_mma(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s);
+cudaError_t launch_attn_fwd_mma_select(const AttnParams& p, const SelectParams& sp, const CUtensorMap* maps,
+                                       cudaStream_t s);
 cudaError_t launch_attn_fwd_tc(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s);
 cudaError_t launch_attn_bwd_mma(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s, bool tc_kv);
 }  // namespace llsa
@@ -196,6 +198,71 @@ bool indices_present(const llsa_desc* d, const llsa_indices* idx, int top) {
   return true;
 }
 
+// The selection launch of level l.
+SelectParams select_params(const llsa_desc* d, const llsa_pyramid* pyr, const llsa_indices* out, int l) {
+  SelectParams p;
+  p.ql = pyr->q[l];
+  p.kl = pyr->k[l];
+  p.parent = (l == d->L) ? nullptr : out->idx[l + 1];
+  p.out = out->idx[l];
+  p.n = n_level(d, l);
+  p.K = k_level(d, l);
+  p.Kp = (l == d->L) ? 0 : k_level(d, l + 1);
+  return p;
+}
+
+int check_select_args(const llsa_desc* d, const llsa_pyramid* pyr, const llsa_indices* out) {
+  if (pyr == nullptr || out == nullptr || !indices_present(d, out, d->L)) return LLSA_ERR_INVALID_ARG;
+  for (int l = 1; l <= d->L; ++l)
+    if (pyr->q[l] == nullptr || pyr->k[l] == nullptr) return LLSA_ERR_INVALID_ARG;
+  return LLSA_OK;
+}
+
+enum class FwdPath { kSimt, kTc, kMma };
+
+struct FwdPlan {
+  AttnParams p;
+  CUtensorMap maps[3];
+  FwdPath path;
+};
+
+// Every check of the forward (and its tensor maps), before anything launches.
+int plan_fwd(const llsa_desc* desc, const void* q, const void* k, const void* v, const llsa_pyramid* pyr,
+             const llsa_indices* idx, void* o, float* lse, int32_t* dev_status, FwdPlan& f) {
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || lse == nullptr ||
+      idx == nullptr || pyr == nullptr)
+    return LLSA_ERR_INVALID_ARG;
+  if (!indices_present(desc, idx, key_top(desc)) || !coarse_kv_present(desc, pyr)) return LLSA_ERR_INVALID_ARG;
+  fill_attn_common(f.p, desc, q, k, v, pyr, idx);
+  f.p.out = o;
+  f.p.lse = lse;
+  f.p.status = dev_status;
+  if (desc->dtype == LLSA_F32) {
+    f.path = FwdPath::kSimt;
+    return LLSA_OK;
+  }
+  // bf16: tensor-core kernels with TMA gathers
+  if (((uintptr_t)o & 15) != 0) return LLSA_ERR_INVALID_ARG;
+  const uint64_t rows = (uint64_t)desc->B * desc->H * desc->N;
+  if (rows > 0x7fffffffULL) return LLSA_ERR_UNSUPPORTED;  // TMA row coordinates are int32
+  const void* srcs[3] = {q, k, v};
+  for (int i = 0; i < 3; ++i) {
+    const int st = make_row_tile_map(&f.maps[i], srcs[i], rows, desc->D);
+    if (st != LLSA_OK) return st;
+  }
+  const bool use_tc = kUseTcForward || (desc->flags & LLSA_FLAG_FWD_TCGEN05) != 0;
+  f.path = (use_tc && desc->D == 64) ? FwdPath::kTc : FwdPath::kMma;  // tcgen05: MMAs into tensor memory
+  return LLSA_OK;
+}
+
+int launch_fwd(const FwdPlan& f, cudaStream_t s) {
+  switch (f.path) {
+    case FwdPath::kSimt: return launch_status(launch_attn_fwd_simt(f.p, LLSA_F32, s));
+    case FwdPath::kTc: return launch_status(launch_attn_fwd_tc(f.p, f.maps, s));
+    default: return launch_status(launch_attn_fwd_mma(f.p, f.maps, s));
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -261,20 +328,11 @@ int llsa_select(const llsa_desc* desc, const llsa_pyramid* pyr, const llsa_indic
                 void* stream) {
   int st = check_desc(desc);
   if (st != LLSA_OK) return st;
-  if (pyr == nullptr || out == nullptr || !indices_present(desc, out, desc->L)) return LLSA_ERR_INVALID_ARG;
-  for (int l = 1; l <= desc->L; ++l)
-    if (pyr->q[l] == nullptr || pyr->k[l] == nullptr) return LLSA_ERR_INVALID_ARG;
+  st = check_select_args(desc, pyr, out);
+  if (st != LLSA_OK) return st;
   const int BH = desc->B * desc->H;
   for (int l = desc->L; l >= 1; --l) {
-    SelectParams p;
-    p.ql = pyr->q[l];
-    p.kl = pyr->k[l];
-    p.parent = (l == desc->L) ? nullptr : out->idx[l + 1];
-    p.out = out->idx[l];
-    p.n = n_level(desc, l);
-    p.K = k_level(desc, l);
-    p.Kp = (l == desc->L) ? 0 : k_level(desc, l + 1);
-    st = launch_status(launch_select_level(p, BH, desc->D, (cudaStream_t)stream));
+    st = launch_status(launch_select_level(select_params(desc, pyr, out, l), BH, desc->D, (cudaStream_t)stream));
     if (st != LLSA_OK) return st;
   }
   return LLSA_OK;
@@ -285,31 +343,34 @@ int llsa_attn_fwd(const llsa_desc* desc, const void* q, const void* k, const voi
                   int32_t* dev_status, void* stream) {
   int st = check_desc(desc);
   if (st != LLSA_OK) return st;
-  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || lse == nullptr ||
-      idx == nullptr || pyr == nullptr)
-    return LLSA_ERR_INVALID_ARG;
-  if (!indices_present(desc, idx, key_top(desc)) || !coarse_kv_present(desc, pyr)) return LLSA_ERR_INVALID_ARG;
-  AttnParams p;
-  fill_attn_common(p, desc, q, k, v, pyr, idx);
-  p.out = o;
-  p.lse = lse;
-  p.status = dev_status;
-  if (desc->dtype == LLSA_F32)
-    return launch_status(launch_attn_fwd_simt(p, desc->dtype, (cudaStream_t)stream));
-  // bf16: tensor-core kernel with TMA gathers
-  if (((uintptr_t)o & 15) != 0) return LLSA_ERR_INVALID_ARG;
-  const uint64_t rows = (uint64_t)desc->B * desc->H * desc->N;
-  if (rows > 0x7fffffffULL) return LLSA_ERR_UNSUPPORTED;  // TMA row coordinates are int32
-  CUtensorMap maps[3];
-  const void* srcs[3] = {q, k, v};
-  for (int i = 0; i < 3; ++i) {
-    st = make_row_tile_map(&maps[i], srcs[i], rows, desc->D);
+  FwdPlan f;
+  st = plan_fwd(desc, q, k, v, pyr, idx, o, lse, dev_status, f);
+  if (st != LLSA_OK) return st;
+  return launch_fwd(f, (cudaStream_t)stream);
+}
+
+int llsa_select_attn_fwd(const llsa_desc* desc, const void* q, const void* k, const void* v,
+                         const llsa_pyramid* pyr, const llsa_indices* idx, void* o, float* lse,
+                         int32_t* dev_status, void* stream) {
+  int st = check_desc(desc);
+  if (st != LLSA_OK) return st;
+  st = check_select_args(desc, pyr, idx);
+  if (st != LLSA_OK) return st;
+  FwdPlan f;
+  st = plan_fwd(desc, q, k, v, pyr, idx, o, lse, dev_status, f);
+  if (st != LLSA_OK) return st;
+  const cudaStream_t s = (cudaStream_t)stream;
+  const int BH = desc->B * desc->H;
+  for (int l = desc->L; l >= 2; --l) {
+    st = launch_status(launch_select_level(select_params(desc, pyr, idx, l), BH, desc->D, s));
     if (st != LLSA_OK) return st;
   }
-  const bool use_tc = kUseTcForward || (desc->flags & LLSA_FLAG_FWD_TCGEN05) != 0;
-  if (use_tc && desc->D == 64)  // tcgen05 MMAs into tensor memory
-    return launch_status(launch_attn_fwd_tc(p, maps, (cudaStream_t)stream));
-  return launch_status(launch_attn_fwd_mma(p, maps, (cudaStream_t)stream));
+  const SelectParams s1 = select_params(desc, pyr, idx, 1);
+  if (f.path == FwdPath::kMma)  // level 1 selected in the forward's prologue
+    return launch_status(launch_attn_fwd_mma_select(f.p, s1, f.maps, s));
+  st = launch_status(launch_select_level(s1, BH, desc->D, s));
+  if (st != LLSA_OK) return st;
+  return launch_fwd(f, s);
 }
 
 size_t llsa_transpose_workspace_bytes(const llsa_desc* desc) {

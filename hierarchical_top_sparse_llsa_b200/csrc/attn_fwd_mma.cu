@@ -18,9 +18,11 @@
 // the softmax is online, in base 2, in fp32 registers.
 
 #include <math.h>
+#include <string.h>
 
 #include "keyset.cuh"
 #include "mma_tiles.cuh"
+#include "select_core.cuh"
 
 namespace llsa {
 
@@ -128,16 +130,26 @@ __device__ __forceinline__ void softmax_tile(float (&s)[2][4], const float (&lw)
   pa[3] = pack_bf16(p[1][2], p[1][3]);
 }
 
-template <int D>
+// kSelect: the CTA first selects I(1) for its 16 query blocks (the level-1
+// step of the hierarchical Top-K, whose 16 sibling queries are exactly this
+// CTA's blocks), writes those rows to p.idx[1] and reads them back below.
+template <int D, bool kSelect>
 __global__ void __launch_bounds__(kFwdWarps * 32)
 attn_fwd_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                    const __grid_constant__ CUtensorMap tv, AttnParams p, int nct) {
+                    const __grid_constant__ CUtensorMap tv, AttnParams p, SelectParams sp, int nct) {
   constexpr int TILE = 32 * D;  // bytes of a 16-row bf16 tile
   constexpr int NT = D / 8;
   constexpr int HALVES = D / 64;
+  static_assert(kFwdWarps * kBPW == kSelQ, "a CTA's query blocks are one selection group");
   extern __shared__ unsigned char smem_raw[];
   unsigned char* sm = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  if constexpr (kSelect) {
+    // the scratch is reused below, partly as TMA destinations
+    select_group<D>(sp, blockIdx.y, blockIdx.x, reinterpret_cast<float*>(sm));
+    fence_proxy_async_smem();
+    __syncthreads();
+  }
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int bh = blockIdx.y;
@@ -175,7 +187,10 @@ attn_fwd_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
     for (int i = 0; i < kBPW; ++i) {
       const int b = wb0 + i;
       const bool on = (b < n1) && lane < K;
-      const int v = on ? p.idx[1][((size_t)bh * n1 + b) * K + lane] : -1;
+      const int32_t* src = p.idx[1] + ((size_t)bh * n1 + b) * K + lane;
+      // rows this CTA has just written: read them from L2, never through the
+      // read-only path
+      const int v = on ? (kSelect ? __ldcg(src) : *src) : -1;
       const bool used = warp_row_used(v, lane, n1, on, flags);
       const unsigned m = __ballot_sync(0xffffffffu, used);
       if (used) flist[i][__popc(m & ((1u << lane) - 1u))] = v;
@@ -353,21 +368,22 @@ attn_fwd_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
   if (lane == 0) report_status(p.status, flags);
 }
 
-template <int D>
-cudaError_t launch_typed(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s) {
+template <int D, bool kSelect>
+cudaError_t launch_typed(const AttnParams& p, const SelectParams& sp, const CUtensorMap* maps, cudaStream_t s) {
   constexpr int TILE = 32 * D;
   const int nct = (p.Kc + 15) / 16;
-  const size_t smem = 1024 + (size_t)kFwdWarps * TILE * (2 + 2 * kStages) + 2 * (size_t)nct * TILE +
-                      nct * 16 * sizeof(float) + kFwdWarps * (2 + kStages) * 8 + nct * 16 * sizeof(int);
-  cudaError_t e = cudaFuncSetAttribute(attn_fwd_mma_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  size_t smem = 1024 + (size_t)kFwdWarps * TILE * (2 + 2 * kStages) + 2 * (size_t)nct * TILE +
+                nct * 16 * sizeof(float) + kFwdWarps * (2 + kStages) * 8 + nct * 16 * sizeof(int);
+  if (kSelect && smem < 1024 + select_scratch_bytes<D>()) smem = 1024 + select_scratch_bytes<D>();
+  auto kern = attn_fwd_mma_kernel<D, kSelect>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(attn_fwd_mma_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
   const int n1 = p.N / kBlock;
   const int per_cta = kFwdWarps * kBPW;
   dim3 grid((n1 + per_cta - 1) / per_cta, p.B * p.H);
-  attn_fwd_mma_kernel<D><<<grid, kFwdWarps * 32, smem, s>>>(maps[0], maps[1], maps[2], p, nct);
+  kern<<<grid, kFwdWarps * 32, smem, s>>>(maps[0], maps[1], maps[2], p, sp, nct);
   return cudaGetLastError();
 }
 
@@ -375,7 +391,16 @@ cudaError_t launch_typed(const AttnParams& p, const CUtensorMap* maps, cudaStrea
 
 // maps: Q, K, V as 2D [B*H*N rows, D cols] bf16, box 16 x 64, 128-byte swizzle.
 cudaError_t launch_attn_fwd_mma(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s) {
-  return (p.D == 64) ? launch_typed<64>(p, maps, s) : launch_typed<128>(p, maps, s);
+  SelectParams none;
+  memset(&none, 0, sizeof(none));
+  return (p.D == 64) ? launch_typed<64, false>(p, none, maps, s) : launch_typed<128, false>(p, none, maps, s);
+}
+
+// The same forward with the level-1 selection in its prologue: sp describes
+// level 1 (parent I(2), out I(1) == p.idx[1]); its query groups are the CTAs.
+cudaError_t launch_attn_fwd_mma_select(const AttnParams& p, const SelectParams& sp, const CUtensorMap* maps,
+                                       cudaStream_t s) {
+  return (p.D == 64) ? launch_typed<64, true>(p, sp, maps, s) : launch_typed<128, true>(p, sp, maps, s);
 }
 
 }  // namespace llsa

@@ -178,6 +178,24 @@ LLSA_API int llsa_attn_fwd(const llsa_desc* desc, const void* q, const void* k, 
                   int32_t* dev_status, void* stream);
 
 /*
+ * llsa_select_attn_fwd - llsa_select followed by llsa_attn_fwd, with the
+ * level-1 step of the selection done inside the forward kernel (each of its
+ * CTAs owns the 16 sibling query blocks of one level-2 token, which is
+ * exactly one level-1 selection group), so I(1) is not read back from memory
+ * by a separate launch.  The paper's kernels run the two steps separately;
+ * the fusion is this library's.
+ *   Arguments as the two calls take them: pyr holds q[l], k[l] for l = 1..L
+ *   and k[l], v[l] for l = 2..Lc; idx: I(1..L), all written (as llsa_select
+ *   writes them; the backward needs them).  Results are identical to the two
+ *   calls made one after the other.  The bf16 warp-MMA forward fuses; with
+ *   fp32 or LLSA_FLAG_FWD_TCGEN05 the level-1 selection runs as its own
+ *   launch before the forward.
+ */
+LLSA_API int llsa_select_attn_fwd(const llsa_desc* desc, const void* q, const void* k, const void* v,
+                                  const llsa_pyramid* pyr, const llsa_indices* idx, void* o, float* lse,
+                                  int32_t* dev_status, void* stream);
+
+/*
  * llsa_transpose_workspace_bytes - device scratch size that
  * llsa_index_transpose needs for desc (0 on an invalid desc): per level,
  * B*H*nchunk*N_l int32 counts with nchunk <= 32 row chunks.

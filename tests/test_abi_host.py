@@ -78,8 +78,32 @@ def test_null_buffers_are_rejected(lib):
     assert llsa.llsa_select(d, pyr, ind, check=False) == llsa.ERR_INVALID_ARG
     assert llsa.llsa_attn_fwd(d, 256, 256, 256, pyr, ind, 256, 256, check=False) == llsa.ERR_INVALID_ARG
     assert llsa.llsa_index_transpose(d, ind, csr, 256, 1 << 40, check=False) == llsa.ERR_INVALID_ARG
+    assert llsa.llsa_select_attn_fwd(d, 256, 256, 256, pyr, ind, 256, 256, check=False) == llsa.ERR_INVALID_ARG
     with pytest.raises(llsa.LlsaError):
         llsa.llsa_select(d, pyr, ind)
+
+
+def test_select_attn_fwd_checks_both_halves_before_launch(lib):
+    d = _desc()
+    pyr, ind = llsa.LlsaPyramid(), llsa.LlsaIndices()
+    for l in range(1, 4):
+        pyr.q[l] = pyr.k[l] = ind.idx[l] = 256
+        if l >= 2:
+            pyr.v[l] = 256
+    # the selection needs Q(1): missing, it is an argument error
+    pyr.q[1] = 0
+    assert llsa.llsa_select_attn_fwd(d, 256, 256, 256, pyr, ind, 256, 256, check=False) == llsa.ERR_INVALID_ARG
+    pyr.q[1] = 256
+    # the forward needs V(2): missing, it is an argument error
+    pyr.v[2] = 0
+    assert llsa.llsa_select_attn_fwd(d, 256, 256, 256, pyr, ind, 256, 256, check=False) == llsa.ERR_INVALID_ARG
+    pyr.v[2] = 256
+    # bf16 output not 16-byte aligned
+    assert llsa.llsa_select_attn_fwd(d, 256, 256, 256, pyr, ind, 264, 256, check=False) == llsa.ERR_INVALID_ARG
+    # I(3) is needed by the selection even when the depth leaves level 3 out
+    d.enrich_levels = 1
+    ind.idx[3] = 0
+    assert llsa.llsa_select_attn_fwd(d, 256, 256, 256, pyr, ind, 264, 256, check=False) == llsa.ERR_INVALID_ARG
 
 
 def test_workspace_size_and_checks(lib):
