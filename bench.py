@@ -54,9 +54,11 @@ def load_peaks():
     return p
 
 
-def algorithmic_work(w: workloads.Workload) -> dict:
+def algorithmic_work(w: workloads.Workload, resid: bool = False) -> dict:
     """Algorithmic bytes and FLOPs of one pass of each stage (no re-reads,
-    no gathers counted).  es = bytes per element of Q/K/V/O/dO/dQ/dK/dV."""
+    no gathers counted).  es = bytes per element of Q/K/V/O/dO/dQ/dK/dV.
+    resid: the forward also writes the bf16 residual of O and the backward
+    reads it (llsa_attn_fwd_res / llsa_attn_bwd_res)."""
     es = 2 if w.dtype == "bf16" else 4
     BH, N, D, K, L = w.B * w.H, w.N, w.D, w.topk, w.L
     fine = BH * N * D * es
@@ -81,6 +83,9 @@ def algorithmic_work(w: workloads.Workload) -> dict:
                       "flops": 0, "bound": "hbm"},
         "bwd": {"bytes": 8 * fine + 2 * BH * N * 4, "flops": 10 * D * pairs, "bound": "hbm"},
     }
+    if resid and w.dtype == "bf16":
+        work["fwd"]["bytes"] += fine
+        work["bwd"]["bytes"] += fine
     return work
 
 
@@ -410,6 +415,8 @@ def run_ours(args, rank, world, local_rank):
     st = bufs.status.data_ptr()
 
     fuse = args.fuse_select
+    resid = not args.no_residual and w.dtype == "bf16" and not args.fwd_tcgen05 and not fuse
+    o_res = torch.empty_like(o) if resid else None
 
     def step(tin, ev=None, sh=sh):
         # ev given: the stages as separate calls with events between them;
@@ -428,7 +435,12 @@ def run_ours(args, rank, world, local_rank):
             llsa.llsa_select(desc, bufs.pyramid, bufs.indices, sh)
             if ev is not None:
                 ev[2].record(stream)
-            llsa.llsa_attn_fwd(desc, q, k, v, bufs.pyramid, bufs.indices, o.data_ptr(), lse.data_ptr(), st, sh)
+            if resid:
+                llsa.llsa_attn_fwd_res(desc, q, k, v, bufs.pyramid, bufs.indices, o.data_ptr(), o_res.data_ptr(),
+                                       lse.data_ptr(), st, sh)
+            else:
+                llsa.llsa_attn_fwd(desc, q, k, v, bufs.pyramid, bufs.indices, o.data_ptr(), lse.data_ptr(), st,
+                                   sh)
         if ev is not None:
             ev[3].record(stream)
         if w.backward:
@@ -436,9 +448,14 @@ def run_ours(args, rank, world, local_rank):
             if ev is not None:
                 ev[4].record(stream)
             dq, dk, dv = grads
-            llsa.llsa_attn_bwd(desc, q, k, v, bufs.pyramid, o.data_ptr(), lse.data_ptr(),
-                               tin["do"].data_ptr(), bufs.indices, bufs.csr, dq.data_ptr(),
-                               dk.data_ptr(), dv.data_ptr(), bufs.ws.data_ptr(), bufs.ws_bytes, st, sh)
+            if resid:
+                llsa.llsa_attn_bwd_res(desc, q, k, v, bufs.pyramid, o.data_ptr(), o_res.data_ptr(), lse.data_ptr(),
+                                       tin["do"].data_ptr(), bufs.indices, bufs.csr, dq.data_ptr(),
+                                       dk.data_ptr(), dv.data_ptr(), bufs.ws.data_ptr(), bufs.ws_bytes, st, sh)
+            else:
+                llsa.llsa_attn_bwd(desc, q, k, v, bufs.pyramid, o.data_ptr(), lse.data_ptr(),
+                                   tin["do"].data_ptr(), bufs.indices, bufs.csr, dq.data_ptr(),
+                                   dk.data_ptr(), dv.data_ptr(), bufs.ws.data_ptr(), bufs.ws_bytes, st, sh)
             if ev is not None:
                 ev[5].record(stream)
 
@@ -536,7 +553,7 @@ def run_ours(args, rank, world, local_rank):
         return
 
     tokens = w.B * w.N
-    work = algorithmic_work(w)
+    work = algorithmic_work(w, resid)
     hbm = peaks["hbm_gbs"]
     tens = peaks["bf16_tflops_sustained"]
     alu_peak = SMS * FP32_LANES_PER_SM * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12  # TFLOP/s, one op per lane-cycle
@@ -597,6 +614,7 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": nlaunch * args.steps,
         "cuda_graph": graph_note,
         "select_in_fwd": fuse,
+        "o_residual": resid,
         "clocks": sampler.summary() if sampler else None,
     }
     print(json.dumps(line), flush=True)
@@ -620,6 +638,9 @@ def main():
                     help="run the key-major backward pass on the tcgen05 kernel (bf16, D=64)")
     ap.add_argument("--fwd-tcgen05", action="store_true",
                     help="run the forward on the tcgen05 kernel (bf16, D=64)")
+    ap.add_argument("--no-residual", action="store_true",
+                    help="time llsa_attn_fwd + llsa_attn_bwd (two walks of each key list) instead of the "
+                         "_res calls (Delta from the bf16 residual of O)")
     ap.add_argument("--fuse-select", action="store_true",
                     help="time llsa_select_attn_fwd (level-1 selection in the forward's prologue) "
                          "instead of llsa_select + llsa_attn_fwd")

@@ -36,6 +36,8 @@ EXPORTED = (
     "llsa_select",
     "llsa_attn_fwd",
     "llsa_select_attn_fwd",
+    "llsa_attn_fwd_res",
+    "llsa_attn_bwd_res",
     "llsa_transpose_workspace_bytes",
     "llsa_index_transpose",
     "llsa_bwd_workspace_bytes",
@@ -102,6 +104,11 @@ def lib() -> ctypes.CDLL:
             "llsa_attn_bwd": (ctypes.c_int, [P(LlsaDesc), vp, vp, vp, P(LlsaPyramid), vp, vp, vp,
                                              P(LlsaIndices), P(LlsaCsr), vp, vp, vp, vp, ctypes.c_size_t,
                                              vp, vp]),
+            "llsa_attn_fwd_res": (ctypes.c_int, [P(LlsaDesc), vp, vp, vp, P(LlsaPyramid), P(LlsaIndices),
+                                                 vp, vp, vp, vp, vp]),
+            "llsa_attn_bwd_res": (ctypes.c_int, [P(LlsaDesc), vp, vp, vp, P(LlsaPyramid), vp, vp, vp, vp,
+                                                 P(LlsaIndices), P(LlsaCsr), vp, vp, vp, vp, ctypes.c_size_t,
+                                                 vp, vp]),
             "llsa_attn_bwd_noalloc": (ctypes.c_int, [P(LlsaDesc), vp, vp, vp, P(LlsaPyramid), vp, vp, vp,
                                                      P(LlsaIndices), P(LlsaCsr), vp, vp, vp, vp, vp]),
             "llsa_reorder": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
@@ -197,6 +204,20 @@ def llsa_attn_bwd(desc, q, k, v, pyramid, o, lse, dout, indices, csr, dq, dk, dv
     st = lib().llsa_attn_bwd(ctypes.byref(desc), q, k, v, ctypes.byref(pyramid), o, lse, dout,
                              ctypes.byref(indices), ctypes.byref(csr), dq, dk, dv, ws, ws_bytes,
                              dev_status, stream)
+    return _check(st) if check else st
+
+
+def llsa_attn_fwd_res(desc, q, k, v, pyramid, indices, o, o_res, lse, dev_status=None, stream=0, check=True):
+    st = lib().llsa_attn_fwd_res(ctypes.byref(desc), q, k, v, ctypes.byref(pyramid), ctypes.byref(indices),
+                                 o, o_res, lse, dev_status, stream)
+    return _check(st) if check else st
+
+
+def llsa_attn_bwd_res(desc, q, k, v, pyramid, o, o_res, lse, dout, indices, csr, dq, dk, dv, ws, ws_bytes,
+                      dev_status=None, stream=0, check=True):
+    st = lib().llsa_attn_bwd_res(ctypes.byref(desc), q, k, v, ctypes.byref(pyramid), o, o_res, lse, dout,
+                                 ctypes.byref(indices), ctypes.byref(csr), dq, dk, dv, ws, ws_bytes,
+                                 dev_status, stream)
     return _check(st) if check else st
 
 

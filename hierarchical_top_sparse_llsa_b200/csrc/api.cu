@@ -263,6 +263,11 @@ int launch_fwd(const FwdPlan& f, cudaStream_t s) {
   }
 }
 
+int attn_bwd_impl(const llsa_desc* desc, const void* q, const void* k, const void* v, const llsa_pyramid* pyr,
+                  const void* o, const void* o_res, const float* lse, const void* dout,
+                  const llsa_indices* idx, const llsa_csr* csr, void* dq, void* dk, void* dv, void* ws,
+                  size_t ws_bytes, int32_t* dev_status, void* stream);
+
 }  // namespace
 
 extern "C" {
@@ -422,6 +427,44 @@ int llsa_attn_bwd(const llsa_desc* desc, const void* q, const void* k, const voi
                   const llsa_pyramid* pyr, const void* o, const float* lse, const void* dout,
                   const llsa_indices* idx, const llsa_csr* csr, void* dq, void* dk, void* dv,
                   void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
+  return attn_bwd_impl(desc, q, k, v, pyr, o, nullptr, lse, dout, idx, csr, dq, dk, dv, ws, ws_bytes, dev_status,
+                       stream);
+}
+
+int llsa_attn_bwd_res(const llsa_desc* desc, const void* q, const void* k, const void* v,
+                      const llsa_pyramid* pyr, const void* o, const void* o_res, const float* lse,
+                      const void* dout, const llsa_indices* idx, const llsa_csr* csr, void* dq, void* dk,
+                      void* dv, void* ws, size_t ws_bytes, int32_t* dev_status, void* stream) {
+  if (desc != nullptr && desc->dtype == LLSA_BF16 && o_res == nullptr) return LLSA_ERR_INVALID_ARG;
+  return attn_bwd_impl(desc, q, k, v, pyr, o, o_res, lse, dout, idx, csr, dq, dk, dv, ws, ws_bytes, dev_status,
+                       stream);
+}
+
+int llsa_attn_fwd_res(const llsa_desc* desc, const void* q, const void* k, const void* v,
+                      const llsa_pyramid* pyr, const llsa_indices* idx, void* o, void* o_res, float* lse,
+                      int32_t* dev_status, void* stream) {
+  int st = check_desc(desc);
+  if (st != LLSA_OK) return st;
+  if (desc->dtype == LLSA_BF16) {  // fp32: O is not rounded, o_res is not used
+    if (o_res == nullptr || ((uintptr_t)o_res & 15) != 0) return LLSA_ERR_INVALID_ARG;
+    if (kUseTcForward || (desc->flags & LLSA_FLAG_FWD_TCGEN05) != 0)
+      return LLSA_ERR_UNSUPPORTED;  // the residual comes from the warp-MMA kernel
+  }
+  FwdPlan f;
+  st = plan_fwd(desc, q, k, v, pyr, idx, o, lse, dev_status, f);
+  if (st != LLSA_OK) return st;
+  if (f.path == FwdPath::kMma) f.p.o_res = o_res;
+  return launch_fwd(f, (cudaStream_t)stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+int attn_bwd_impl(const llsa_desc* desc, const void* q, const void* k, const void* v, const llsa_pyramid* pyr,
+                  const void* o, const void* o_res, const float* lse, const void* dout,
+                  const llsa_indices* idx, const llsa_csr* csr, void* dq, void* dk, void* dv, void* ws,
+                  size_t ws_bytes, int32_t* dev_status, void* stream) {
   int st = check_desc(desc);
   if (st != LLSA_OK) return st;
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || lse == nullptr ||
@@ -455,11 +498,12 @@ int llsa_attn_bwd(const llsa_desc* desc, const void* q, const void* k, const voi
   p.dk = dk;
   p.dv = dv;
   p.status = dev_status;
-  if (desc->dtype == LLSA_F32)
+  if (desc->dtype == LLSA_F32)  // O is stored unrounded: a residual is not used
     return launch_status(launch_attn_bwd_simt(p, desc->dtype, (cudaStream_t)stream));
   // bf16: tensor-core kernels with TMA gathers
-  if ((((uintptr_t)dq | (uintptr_t)dk | (uintptr_t)dv | (uintptr_t)lse) & 15) != 0)
+  if ((((uintptr_t)dq | (uintptr_t)dk | (uintptr_t)dv | (uintptr_t)lse | (uintptr_t)o_res) & 15) != 0)
     return LLSA_ERR_INVALID_ARG;  // 16-byte stores and bulk copies
+  p.o_res = const_cast<void*>(o_res);
   const uint64_t rows = (uint64_t)desc->B * desc->H * desc->N;
   if (rows > 0x7fffffffULL) return LLSA_ERR_UNSUPPORTED;  // TMA row coordinates are int32
   CUtensorMap maps[4];
@@ -472,4 +516,4 @@ int llsa_attn_bwd(const llsa_desc* desc, const void* q, const void* k, const voi
   return launch_status(launch_attn_bwd_mma(p, maps, (cudaStream_t)stream, tc_kv));
 }
 
-}  // extern "C"
+}  // namespace

@@ -89,7 +89,10 @@ __device__ __forceinline__ void ds_rows(float (&P)[2][4], const float (&dp)[2][4
   }
 }
 
-template <int D>
+// kResid: Delta_i = dO_i . (O_i + R_i) from the forward's bf16 rounding
+// residual R of O (together about 16 mantissa bits beyond bf16), read at the
+// start, so the key list is walked once instead of twice.
+template <int D, bool kResid>
 __global__ void __launch_bounds__(kQWarps * 32)
 bwd_q_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                  const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
@@ -184,7 +187,7 @@ bwd_q_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
     clw[e] = (e < nc) ? p.logw[clist[e] >> 24] * kLog2e : -INFINITY;
 
   const size_t rowbase = (size_t)bh * p.N;
-  const int ntiles = 2 * nf;  // the fine key list is walked twice
+  const int ntiles = kResid ? nf : 2 * nf;  // without the residual the fine key list is walked twice
   auto issue = [&](int r) {
     if (lane == 0) {
       const int blk = flist[r % nf];
@@ -220,10 +223,39 @@ bwd_q_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
   const float sc2 = p.scale * kLog2e;
   const float zero_lw[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
   if (active) {
-    ok = mbar_wait_bounded(bar0, 0);
+    ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar0, 0));  // warp-uniform before the shuffles
     const size_t tok0 = rowbase + (size_t)b * 16 + g;
     lse_g = p.lse_in[tok0] * kLog2e;
     lse_g8 = p.lse_in[tok0 + 8] * kLog2e;
+    if constexpr (kResid) {
+      if (ok) {
+        // dO from this warp's tile (swizzled), O and its residual from memory;
+        // lane (g, t) sums columns 8nt + 2t, +1 of rows g and g+8
+        const bf16* Og = static_cast<const bf16*>(p.o);
+        const bf16* Rg = static_cast<const bf16*>(p.o_res);
+        float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          uint32_t d0, d1;
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(d0) : "r"(dot + swz(g, nt) + 4 * t));
+          asm volatile("ld.shared.u32 %0, [%1];" : "=r"(d1) : "r"(dot + swz(g + 8, nt) + 4 * t));
+          const uint32_t o0 = *reinterpret_cast<const uint32_t*>(Og + tok0 * D + 8 * nt + 2 * t);
+          const uint32_t o1 = *reinterpret_cast<const uint32_t*>(Og + (tok0 + 8) * D + 8 * nt + 2 * t);
+          const uint32_t r0 = *reinterpret_cast<const uint32_t*>(Rg + tok0 * D + 8 * nt + 2 * t);
+          const uint32_t r1 = *reinterpret_cast<const uint32_t*>(Rg + (tok0 + 8) * D + 8 * nt + 2 * t);
+          a0 = fmaf(bf16x2_lo(d0), bf16x2_lo(o0) + bf16x2_lo(r0), a0);
+          a0 = fmaf(bf16x2_hi(d0), bf16x2_hi(o0) + bf16x2_hi(r0), a0);
+          a1 = fmaf(bf16x2_lo(d1), bf16x2_lo(o1) + bf16x2_lo(r1), a1);
+          a1 = fmaf(bf16x2_hi(d1), bf16x2_hi(o1) + bf16x2_hi(r1), a1);
+        }
+        a0 += __shfl_xor_sync(0xffffffffu, a0, 1);
+        a0 += __shfl_xor_sync(0xffffffffu, a0, 2);
+        a1 += __shfl_xor_sync(0xffffffffu, a1, 1);
+        a1 += __shfl_xor_sync(0xffffffffu, a1, 2);
+        delta_g = a0;
+        delta_g8 = a1;
+      }
+    }
     // Both sweeps walk the ring tiles 0..2nf-1 with one software pipeline:
     // S and dP of tile r+1 are issued before the elementwise work of tile r.
     float dp0 = 0.f, dp1 = 0.f;
@@ -248,7 +280,7 @@ bwd_q_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
       }
       float P[2][4];
       probs_rows(s_cur, zero_lw, sc2, lse_g, lse_g8, P);
-      if (r < nf) {  // sweep 1: Delta
+      if (!kResid && r < nf) {  // sweep 1: Delta
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
           dp0 += P[nt][0] * d_cur[nt][0] + P[nt][1] * d_cur[nt][1];
@@ -298,7 +330,7 @@ bwd_q_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__
           }
       }
     }
-    if (nf == 0 && ok) {  // no fine keys: Delta from the coarse keys alone
+    if (!kResid && nf == 0 && ok) {  // no fine keys: Delta from the coarse keys alone
       for (int ct = 0; ct < ncpad; ++ct) {
         float s[2][4], dpv[2][4], Pc[2][4], lw[2][2];
 #pragma unroll
@@ -688,12 +720,13 @@ cudaError_t launch_typed(const AttnParams& p, const CUtensorMap* maps, cudaStrea
   // pass 1
   const size_t smem1 = 1024 + (size_t)kQWarps * TILE * (2 + 2 * kRing) + 2 * (size_t)nct * TILE +
                        nct * 16 * sizeof(float) + kQWarps * (1 + kRing) * 8 + 2 * nct * 16 * sizeof(int);
-  cudaError_t e = cudaFuncSetAttribute(bwd_q_mma_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
+  auto kern1 = (p.o_res != nullptr) ? bwd_q_mma_kernel<D, true> : bwd_q_mma_kernel<D, false>;
+  cudaError_t e = cudaFuncSetAttribute(kern1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem1);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(bwd_q_mma_kernel<D>, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+  e = cudaFuncSetAttribute(kern1, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
-  bwd_q_mma_kernel<D><<<dim3((n1 + kQWarps - 1) / kQWarps, BH), kQWarps * 32, smem1, s>>>(
-      maps[0], maps[1], maps[2], maps[3], p, nct);
+  kern1<<<dim3((n1 + kQWarps - 1) / kQWarps, BH), kQWarps * 32, smem1, s>>>(maps[0], maps[1], maps[2], maps[3], p,
+                                                                            nct);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   // pass 2

@@ -347,11 +347,21 @@ attn_fwd_mma_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constan
     const float i0 = l0 > 0.f ? 1.f / l0 : 0.f;
     const float i1 = l1 > 0.f ? 1.f / l1 : 0.f;
     bf16* O = static_cast<bf16*>(p.out);
+    bf16* R = static_cast<bf16*>(p.o_res);
     const size_t tok0 = rowbase + (size_t)b * 16 + g;
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      *reinterpret_cast<uint32_t*>(O + tok0 * D + 8 * nt + 2 * t) = pack_bf16(o[nt][0] * i0, o[nt][1] * i0);
-      *reinterpret_cast<uint32_t*>(O + (tok0 + 8) * D + 8 * nt + 2 * t) = pack_bf16(o[nt][2] * i1, o[nt][3] * i1);
+      const float a0 = o[nt][0] * i0, a1 = o[nt][1] * i0;  // row g
+      const float c0 = o[nt][2] * i1, c1 = o[nt][3] * i1;  // row g+8
+      const uint32_t h0 = pack_bf16(a0, a1), h1 = pack_bf16(c0, c1);
+      *reinterpret_cast<uint32_t*>(O + tok0 * D + 8 * nt + 2 * t) = h0;
+      *reinterpret_cast<uint32_t*>(O + (tok0 + 8) * D + 8 * nt + 2 * t) = h1;
+      if (R != nullptr) {  // what the bf16 rounding of O left out, itself in bf16
+        *reinterpret_cast<uint32_t*>(R + tok0 * D + 8 * nt + 2 * t) =
+            pack_bf16(a0 - bf16x2_lo(h0), a1 - bf16x2_hi(h0));
+        *reinterpret_cast<uint32_t*>(R + (tok0 + 8) * D + 8 * nt + 2 * t) =
+            pack_bf16(c0 - bf16x2_lo(h1), c1 - bf16x2_hi(h1));
+      }
     }
     if (t == 0) {
       p.lse[tok0] = l0 > 0.f ? (st.m[0] + log2f(l0)) * kLn2 : -INFINITY;

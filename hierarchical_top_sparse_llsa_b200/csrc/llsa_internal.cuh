@@ -165,6 +165,7 @@ struct AttnParams {
   const int32_t* col[kMaxL + 1];
   float logw[kMaxL + 1];  // ln of the level weights (0 for weight 1)
   void* out;              // O (fwd)
+  void* o_res;            // bf16 rounding residual of O: written by the fwd, read by the bwd (null: none)
   float* lse;             // LSE (fwd)
   void* dq;
   void* dk;

@@ -163,6 +163,10 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// The two halves of a packed bf16 pair (pack_bf16 order), widened exactly.
+__device__ __forceinline__ float bf16x2_lo(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf16x2_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
+
 // Byte offset of the 16-byte chunk `j` (0..D/8-1) of row `r` in a tile of
 // 16 rows written by a TMA load with 128-byte swizzle: each 64-column half of
 // the row lives in its own 16 x 128-byte sub-tile (2 KB), and inside it the

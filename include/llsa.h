@@ -196,6 +196,21 @@ LLSA_API int llsa_select_attn_fwd(const llsa_desc* desc, const void* q, const vo
                                   int32_t* dev_status, void* stream);
 
 /*
+ * llsa_attn_fwd_res - llsa_attn_fwd that also writes the rounding residual
+ * of O, for a backward that takes it (llsa_attn_bwd_res).  The paper's
+ * kernels have no counterpart: this is a speed option of this library.
+ *   o_res: [B, H, N, D] bf16, 16-byte aligned, written with
+ *   bf16(O_fp32 - float(o)) element by element, where O_fp32 is the kernel's
+ *   fp32 output before rounding; o + o_res then holds O to about 16 mantissa
+ *   bits.  o and lse are identical to llsa_attn_fwd's.
+ *   dtype LLSA_F32: O is stored unrounded, o_res is not used (may be NULL).
+ *   LLSA_FLAG_FWD_TCGEN05 with bf16 gives LLSA_ERR_UNSUPPORTED.
+ */
+LLSA_API int llsa_attn_fwd_res(const llsa_desc* desc, const void* q, const void* k, const void* v,
+                               const llsa_pyramid* pyr, const llsa_indices* idx, void* o, void* o_res,
+                               float* lse, int32_t* dev_status, void* stream);
+
+/*
  * llsa_transpose_workspace_bytes - device scratch size that
  * llsa_index_transpose needs for desc (0 on an invalid desc): per level,
  * B*H*nchunk*N_l int32 counts with nchunk <= 32 row chunks.
@@ -248,6 +263,23 @@ LLSA_API int llsa_attn_bwd(const llsa_desc* desc, const void* q, const void* k, 
                   const llsa_pyramid* pyr, const void* o, const float* lse, const void* dout,
                   const llsa_indices* idx, const llsa_csr* csr, void* dq, void* dk, void* dv,
                   void* ws, size_t ws_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * llsa_attn_bwd_res - llsa_attn_bwd with Delta_i = dO_i . (o_i + o_res_i)
+ * (fp32 sums) from the residual that llsa_attn_fwd_res wrote, instead of
+ * Delta_i = sum_j P_ij (dO_i . v_j) over the key set: the query-major pass
+ * then walks each key list once instead of twice.  Within the same error bar
+ * as llsa_attn_bwd, not bit-identical to it.
+ *   o_res: bf16 [B, H, N, D], 16-byte aligned (NULL with bf16 gives
+ *   LLSA_ERR_INVALID_ARG).  dtype LLSA_F32: o_res is not used (may be NULL;
+ *   O itself is unrounded) and the call equals llsa_attn_bwd.
+ *   Other arguments as llsa_attn_bwd.
+ */
+LLSA_API int llsa_attn_bwd_res(const llsa_desc* desc, const void* q, const void* k, const void* v,
+                               const llsa_pyramid* pyr, const void* o, const void* o_res, const float* lse,
+                               const void* dout, const llsa_indices* idx, const llsa_csr* csr, void* dq,
+                               void* dk, void* dv, void* ws, size_t ws_bytes, int32_t* dev_status,
+                               void* stream);
 
 /*
  * llsa_attn_bwd_noalloc - llsa_attn_bwd for callers that cannot allocate.

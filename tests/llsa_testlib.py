@@ -59,8 +59,10 @@ def assert_close(got, want, dtype: str, what: str):
 
 
 def run_gpu(B, H, N, D, L, topk, dtype, inputs, level_w=None, ext_idx=None, bwd=True,
-            device="cuda", flags=0, enrich=0, topk_l=None):
-    """The whole path through the C ABI.  Returns numpy copies of everything."""
+            device="cuda", flags=0, enrich=0, topk_l=None, resid=False):
+    """The whole path through the C ABI.  Returns numpy copies of everything.
+    resid: run llsa_attn_fwd_res / llsa_attn_bwd_res (Delta from the O
+    residual) instead of llsa_attn_fwd / llsa_attn_bwd."""
     import torch
 
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
@@ -82,18 +84,33 @@ def run_gpu(B, H, N, D, L, topk, dtype, inputs, level_w=None, ext_idx=None, bwd=
             bufs.idx[l].copy_(torch.from_numpy(np.ascontiguousarray(I, dtype=np.int32)))
     o = torch.empty_like(t["q"])
     lse = torch.empty(B, H, N, dtype=torch.float32, device=device)
-    llsa.llsa_attn_fwd(desc, t["q"].data_ptr(), t["k"].data_ptr(), t["v"].data_ptr(), bufs.pyramid,
-                       bufs.indices, o.data_ptr(), lse.data_ptr(), st, stream)
+    o_res = torch.full_like(o, float("nan")) if resid and dtype == "bf16" else None
+    if resid:
+        llsa.llsa_attn_fwd_res(desc, t["q"].data_ptr(), t["k"].data_ptr(), t["v"].data_ptr(), bufs.pyramid,
+                               bufs.indices, o.data_ptr(), o_res.data_ptr() if o_res is not None else None,
+                               lse.data_ptr(), st, stream)
+    else:
+        llsa.llsa_attn_fwd(desc, t["q"].data_ptr(), t["k"].data_ptr(), t["v"].data_ptr(), bufs.pyramid,
+                           bufs.indices, o.data_ptr(), lse.data_ptr(), st, stream)
     if bwd:
         llsa.llsa_index_transpose(desc, bufs.indices, bufs.csr, bufs.tr_ws.data_ptr(), bufs.tr_ws_bytes, st, stream)
         dq, dk, dv = torch.empty_like(o), torch.empty_like(o), torch.empty_like(o)
-        llsa.llsa_attn_bwd(desc, t["q"].data_ptr(), t["k"].data_ptr(), t["v"].data_ptr(), bufs.pyramid,
-                           o.data_ptr(), lse.data_ptr(), t["do"].data_ptr(), bufs.indices, bufs.csr,
-                           dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), bufs.ws.data_ptr(),
-                           bufs.ws_bytes, st, stream)
+        if resid:
+            llsa.llsa_attn_bwd_res(desc, t["q"].data_ptr(), t["k"].data_ptr(), t["v"].data_ptr(), bufs.pyramid,
+                                   o.data_ptr(), o_res.data_ptr() if o_res is not None else None,
+                                   lse.data_ptr(), t["do"].data_ptr(), bufs.indices, bufs.csr,
+                                   dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), bufs.ws.data_ptr(),
+                                   bufs.ws_bytes, st, stream)
+        else:
+            llsa.llsa_attn_bwd(desc, t["q"].data_ptr(), t["k"].data_ptr(), t["v"].data_ptr(), bufs.pyramid,
+                               o.data_ptr(), lse.data_ptr(), t["do"].data_ptr(), bufs.indices, bufs.csr,
+                               dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), bufs.ws.data_ptr(),
+                               bufs.ws_bytes, st, stream)
     torch.cuda.synchronize()
     out["idx"] = {l: bufs.idx[l].cpu().numpy() for l in bufs.idx}
     out["O"] = o.float().cpu().numpy()
+    if o_res is not None:
+        out["O_res"] = o_res.float().cpu().numpy()
     out["LSE"] = lse.cpu().numpy()
     if bwd:
         out["row_ptr"] = {l: bufs.row_ptr[l].cpu().numpy() for l in bufs.row_ptr}

@@ -223,3 +223,20 @@ def test_topk_per_level_sizes_and_checks(lib):
     assert llsa.llsa_select(bad, pyr, ind, check=False) == llsa.ERR_INVALID_ARG
     bad.topk_l[2] = 40
     assert llsa.llsa_select(bad, pyr, ind, check=False) == llsa.ERR_UNSUPPORTED
+
+
+def test_residual_calls_check_arguments(lib):
+    d = _desc()
+    pyr, ind, csr = llsa.LlsaPyramid(), llsa.LlsaIndices(), llsa.LlsaCsr()
+    for l in range(1, 4):
+        pyr.q[l] = pyr.k[l] = ind.idx[l] = csr.row_ptr[l] = csr.col[l] = 256
+        if l >= 2:
+            pyr.v[l] = 256
+    # bf16 without a residual buffer, or a misaligned one
+    assert llsa.llsa_attn_bwd_res(d, 256, 256, 256, pyr, 256, None, 256, 256, ind, csr, 256, 256, 256,
+                                  256, 1 << 40, check=False) == llsa.ERR_INVALID_ARG
+    assert llsa.llsa_attn_fwd_res(d, 256, 256, 256, pyr, ind, 256, None, 256, check=False) == llsa.ERR_INVALID_ARG
+    assert llsa.llsa_attn_fwd_res(d, 256, 256, 256, pyr, ind, 264, 256, 256, check=False) == llsa.ERR_INVALID_ARG
+    ws = llsa.llsa_bwd_workspace_bytes(d)
+    assert llsa.llsa_attn_bwd_res(d, 256, 256, 256, pyr, 256, 264, 256, 256, ind, csr, 256, 256, 256,
+                                  256, ws - 1, check=False) == llsa.ERR_WORKSPACE
