@@ -199,6 +199,74 @@ def reorder_rate(torch, llsa, w, dev, src, hbm_gbs, iters=10):
             "tensor": f"[{w.B}, {w.H}, {w.N}, {w.D}] {str(src.dtype).replace('torch.', '')}"}
 
 
+def gathered_select_bytes(w: workloads.Workload) -> int:
+    """Candidate K(l) rows the selection loads (fp32), once per group of 16
+    sibling queries (they share one candidate list), plus the Q(l) rows."""
+    BH, D, L = w.B * w.H, w.D, w.L
+    keff = w.k_eff()
+    total = 0
+    for l in range(1, L + 1):
+        n = w.n_level(l)
+        groups = -(-n // 16)
+        cand = n if l == L else 16 * keff[l + 1]
+        total += BH * (groups * cand + n) * D * 4
+    return total
+
+
+def transpose_graph_rate(torch, llsa, desc, bufs, dev, hbm_gbs, compulsory, repeats=20):
+    """The index transpose as `repeats` back-to-back calls in one CUDA graph
+    (launch gaps removed): ms per call and GB/s of its compulsory bytes."""
+    s = torch.cuda.Stream(dev)
+    s.wait_stream(torch.cuda.current_stream(dev))
+    g = torch.cuda.CUDAGraph()
+    call = lambda: llsa.llsa_index_transpose(desc, bufs.indices, bufs.csr, bufs.tr_ws.data_ptr(), bufs.tr_ws_bytes,
+                                             None, s.cuda_stream)
+    with torch.cuda.stream(s):
+        call()
+    torch.cuda.synchronize()
+    with torch.cuda.graph(g, stream=s):
+        for _ in range(repeats):
+            call()
+    g.replay()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / repeats
+    gbs = compulsory / (ms * 1e-3) / 1e9
+    del g
+    return {"ms": round(ms, 4), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm_gbs, 4),
+            "repeats_in_graph": repeats}
+
+
+def transpose_512_k32(torch, llsa, dev, hbm_gbs):
+    """The index transpose at the 512x512-pixel, K = 32 shape (B = 1, H = 8,
+    N = 262144, D = 128, L = 4: 36 MB of lists), where its compulsory bytes
+    are large enough to measure bandwidth.  Its indices come from the path's
+    own pool and selection on device-drawn N(0, 1) inputs (only the index
+    pattern matters here)."""
+    w = workloads.WORKLOADS["img512_k32_bf16"]
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed)
+    x = [torch.randn(w.B, w.H, w.N, w.D, device=dev, dtype=torch.bfloat16, generator=g) for _ in range(3)]
+    desc = llsa.make_desc(w.B, w.H, w.N, w.D, w.L, w.topk, llsa.BF16)
+    bufs = llsa.LlsaBuffers(desc, dev, with_bwd=True)
+    sh = torch.cuda.current_stream(dev).cuda_stream
+    llsa.llsa_pool(desc, x[0].data_ptr(), x[1].data_ptr(), x[2].data_ptr(), bufs.pyramid, sh)
+    llsa.llsa_select(desc, bufs.pyramid, bufs.indices, sh)
+    torch.cuda.synchronize()
+    del x
+    work = algorithmic_work(w)["transpose"]["bytes"]
+    rec = transpose_graph_rate(torch, llsa, desc, bufs, dev, hbm_gbs, work)
+    rec["workload"] = f"{w.name}: N={w.N}, B={w.B}, H={w.H}, L={w.L}, K={w.topk}"
+    del bufs
+    torch.cuda.empty_cache()
+    return rec
+
+
 def select_scaling(args):
     """Selection cost against N: hierarchical (the levels of the path's
     workloads: L = 3 up to 256x256 pixels, 4 at 512x512) and single-level (L = 1: every query block scores every
@@ -598,10 +666,14 @@ def run_ours(args, rank, world, local_rank):
         wk = work[n]
         gbs = wk["bytes"] / (t_ms * 1e-3) / 1e9
         tfl = wk["flops"] / (t_ms * 1e-3) / 1e12
-        stages[n] = {"ms": round(t_ms, 4), "GB/s": round(gbs, 1), "TFLOP/s": round(tfl, 2),
-                     "frac_hbm": round(gbs / hbm, 4), "frac_bf16_tensor": round(tfl / tens, 4)}
+        stages[n] = {"ms": round(t_ms, 4), "tokens/s": round(tokens / (t_ms * 1e-3)), "GB/s": round(gbs, 1),
+                     "TFLOP/s": round(tfl, 2), "frac_hbm": round(gbs / hbm, 4),
+                     "frac_bf16_tensor": round(tfl / tens, 4)}
         if wk["bound"] == "alu":
             stages[n]["frac_fp32_alu"] = round(tfl / alu_peak, 4)
+        # the binding roofline: the slower of its memory and its arithmetic floor
+        t_floor = max(wk["bytes"] / (hbm * 1e9), wk["flops"] / ((alu_peak if wk["bound"] == "alu" else tens) * 1e12))
+        stages[n]["frac_binding"] = round(t_floor / (t_ms * 1e-3), 4)
     dom = max(stage_ms, key=stage_ms.get)
     wk = work[dom]
     if wk["bound"] == "alu":
@@ -619,6 +691,10 @@ def run_ours(args, rank, world, local_rank):
     roof["kernel"] = f"llsa_{'attn_' if dom in ('fwd', 'bwd') else ''}{dom} ({launches_per_step(w.L)[dom]} launches)"
     roof["peak_source"] = f"{peaks['source']} (MEASURED_PEAKS.json)" if peaks["source"] == "measured" else "fallback"
     reorder = reorder_rate(torch, llsa, w, dev, t_in["q"], peaks["hbm_gbs"])
+    tr_graph = None
+    if w.backward and not args.no_transpose_graph:
+        tr_graph = {"headline": transpose_graph_rate(torch, llsa, desc, bufs, dev, hbm, work["transpose"]["bytes"])}
+        tr_graph["img512_k32"] = transpose_512_k32(torch, llsa, dev, hbm)
     dense = None
     if w.backward and not args.no_dense:
         dense = dense_reference(torch, w, dev)
@@ -641,6 +717,8 @@ def run_ours(args, rank, world, local_rank):
         "fwd_bwd_ms": attn_ms,
         "fwd_bwd_frac_bf16_tensor": attn_flops / (attn_ms * 1e-3) / 1e12 / tens,
         "selection_GBps": (work["pool"]["bytes"] + work["select"]["bytes"]) / (sel_ms * 1e-3) / 1e9,
+        "select_gathered_GBps": gathered_select_bytes(w) / (stage_ms["select"] * 1e-3) / 1e9,
+        "transpose_graph": tr_graph,
         "roofline": roof,
         "cpu_baseline": cpu,
         "dense_reference": dense,
@@ -675,6 +753,8 @@ def main():
                     help="run the key-major backward pass on the tcgen05 kernel (bf16, D=64)")
     ap.add_argument("--fwd-tcgen05", action="store_true",
                     help="run the forward on the tcgen05 kernel (bf16, D=64)")
+    ap.add_argument("--no-transpose-graph", action="store_true",
+                    help="skip the index transpose timed as back-to-back calls in a CUDA graph")
     ap.add_argument("--no-residual", action="store_true",
                     help="time llsa_attn_fwd + llsa_attn_bwd (two walks of each key list) instead of the "
                          "_res calls (Delta from the bf16 residual of O)")

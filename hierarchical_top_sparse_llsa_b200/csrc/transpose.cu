@@ -16,8 +16,9 @@
 //           row_ptr, and -1 in the unused tail of col;
 //   fill    one CTA per chunk: the cursors row_ptr[c] + first slot are staged
 //           in shared memory, then one warp walks the chunk's rows in order,
-//           lanes that share a key in one step ranked by __match_any_sync,
-//           and writes each query at its key's cursor.
+//           lanes that share a key in one step ranked by __match_any_sync
+//           and advanced by one shared-memory atomic per group, and writes
+//           each query at its key's cursor.
 // Chunks are filled in row order from the slots the prefix gave them, so
 // every key's list comes out ascending and the result is deterministic.
 // Entries are screened with the same used-entry rule as the attention
@@ -34,7 +35,7 @@ constexpr int kPrefixThreads = 256;
 constexpr int kPrefixKeys = 4 * kPrefixThreads;  // keys per prefix CTA
 constexpr int kScanThreads = 1024;
 constexpr int kFillThreads = 256;  // all stage the cursors; warp 0 fills
-constexpr int kMaxChunks = 32;     // row chunks per (level, b, h); see transpose_chunking
+constexpr int kMaxChunks = 128;    // row chunks per (level, b, h); see transpose_chunking
 constexpr int kRangeKeys = 8192;   // keys per shared-memory histogram / cursor range
 constexpr int kBatch = 8;          // row steps whose index loads are in flight together
 
@@ -256,14 +257,20 @@ tr_fill_kernel(TransposeParams p) {
           peers[i] = __match_any_sync(0xffffffffu, key[i]);
           rank[i] = __popc(peers[i] & ((1u << lane) - 1u));  // lower lanes hold lower rows
         }
-        // the cursor updates run in step order
+        // The cursor updates run in step order: the highest lane of each group
+        // of lanes sharing a key takes the group's slots with one shared-memory
+        // atomic (one warp instruction per step, so same-key atomics of
+        // consecutive steps are applied in step order) and hands the base to
+        // its group by a shuffle.  No warp barrier is needed between steps, so
+        // none waits for the scattered stores into col.
 #pragma unroll
         for (int i = 0; i < kBatch; ++i) {
           const int q = rb + i * rl.rows_per_step + rl.sub;
-          if (key[i] >= 0) col[cur[key[i]] + rank[i]] = q;
-          __syncwarp();
-          if (key[i] >= 0 && lane == 31 - __clz(peers[i])) cur[key[i]] += __popc(peers[i]);
-          __syncwarp();
+          const int leader = 31 - __clz(peers[i]);
+          int base = 0;
+          if (key[i] >= 0 && lane == leader) base = atomicAdd(&cur[key[i]], __popc(peers[i]));
+          base = __shfl_sync(0xffffffffu, base, leader);
+          if (key[i] >= 0) col[base + rank[i]] = q;
         }
 #pragma unroll
         for (int i = 0; i < kBatch; ++i) cb[i] = nb[i];
@@ -275,10 +282,12 @@ tr_fill_kernel(TransposeParams p) {
 
 }  // namespace
 
-// Rows per chunk for a level of n query rows: at most kMaxChunks chunks, at
-// least 64 rows each (the workspace holds nchunk * n counts per (b, h)).
+// Rows per chunk for a level of n query rows: 128 rows per chunk (one warp
+// fills a chunk in row order, so the chunk length bounds the fill's critical
+// path), at most kMaxChunks chunks (the workspace holds nchunk * n counts per
+// (b, h)).
 void transpose_chunking(int n, int* nchunk, int* rows) {
-  int c = (n + 63) / 64;
+  int c = (n + 127) / 128;
   if (c > kMaxChunks) c = kMaxChunks;
   if (c < 1) c = 1;
   *rows = (n + c - 1) / c;

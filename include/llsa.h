@@ -213,7 +213,7 @@ LLSA_API int llsa_attn_fwd_res(const llsa_desc* desc, const void* q, const void*
 /*
  * llsa_transpose_workspace_bytes - device scratch size that
  * llsa_index_transpose needs for desc (0 on an invalid desc): per level,
- * B*H*nchunk*N_l int32 counts with nchunk <= 32 row chunks.
+ * B*H*nchunk*N_l int32 counts with nchunk <= 128 row chunks.
  */
 LLSA_API size_t llsa_transpose_workspace_bytes(const llsa_desc* desc);
 

@@ -128,12 +128,12 @@ def test_workspace_size_and_checks(lib):
 
 
 def _transpose_ws_bytes(B, H, N, L):
-    # per level: nchunk row chunks (at most 32, at least 64 rows each), one
+    # per level: nchunk row chunks (128 rows each, at most 128 chunks), one
     # int32 count per (b, h, chunk, key), each level 256-byte aligned
     total = 0
     for l in range(1, L + 1):
         n = N // 16**l
-        c = min(32, max(1, (n + 63) // 64))
+        c = min(128, max(1, (n + 127) // 128))
         rows = (n + c - 1) // c
         c = (n + rows - 1) // rows
         total += (B * H * c * n * 4 + 255) // 256 * 256
