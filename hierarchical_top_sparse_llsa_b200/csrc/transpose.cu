@@ -254,8 +254,14 @@ tr_fill_kernel(TransposeParams p) {
           const int c = cb[i];
           const bool u = warp_row_used(c, rl.slot, n, rl.on && q < r1, dummy, K);
           key[i] = (u && c >= k0 && c < k0 + len) ? c - k0 : -1 - lane;  // -1 - lane matches nobody
-          peers[i] = __match_any_sync(0xffffffffu, key[i]);
-          rank[i] = __popc(peers[i] & ((1u << lane) - 1u));  // lower lanes hold lower rows
+          if (rl.rows_per_step == 1) {
+            // one row per step: its used entries are distinct keys
+            peers[i] = 1u << lane;
+            rank[i] = 0;
+          } else {
+            peers[i] = __match_any_sync(0xffffffffu, key[i]);
+            rank[i] = __popc(peers[i] & ((1u << lane) - 1u));  // lower lanes hold lower rows
+          }
         }
         // The cursor updates run in step order: the highest lane of each group
         // of lanes sharing a key takes the group's slots with one shared-memory
@@ -269,7 +275,7 @@ tr_fill_kernel(TransposeParams p) {
           const int leader = 31 - __clz(peers[i]);
           int base = 0;
           if (key[i] >= 0 && lane == leader) base = atomicAdd(&cur[key[i]], __popc(peers[i]));
-          base = __shfl_sync(0xffffffffu, base, leader);
+          if (rl.rows_per_step > 1) base = __shfl_sync(0xffffffffu, base, leader);
           if (key[i] >= 0) col[base + rank[i]] = q;
         }
 #pragma unroll
