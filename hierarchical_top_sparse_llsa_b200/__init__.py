@@ -74,6 +74,11 @@ class LlsaCsr(ctypes.Structure):
     _fields_ = [("row_ptr", _PtrArr), ("col", _PtrArr)]
 
 
+# llsa_version() of the library whose struct layouts (llsa_desc above) this
+# binding mirrors
+ABI_VERSION = 200
+
+
 class LlsaError(RuntimeError):
     """A host status other than LLSA_OK."""
 
@@ -120,6 +125,9 @@ def lib() -> ctypes.CDLL:
             fn = getattr(L, name)
             fn.restype = res
             fn.argtypes = args
+        if L.llsa_version() != ABI_VERSION:  # the structs above would not match its layout
+            raise LlsaError(f"{LIB_PATH} is version {L.llsa_version()}, this binding expects {ABI_VERSION}: "
+                            "rebuild the CUDA library")
         _lib = L
     return _lib
 

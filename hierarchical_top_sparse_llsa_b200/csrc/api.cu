@@ -272,7 +272,7 @@ int attn_bwd_impl(const llsa_desc* desc, const void* q, const void* k, const voi
 
 extern "C" {
 
-int llsa_version(void) { return 100; }
+int llsa_version(void) { return 200; }  // 0.2.0: llsa_desc gained enrich_levels and topk_l
 
 int llsa_reorder(int B, int H, int img_h, int img_w, int D, int dtype, const void* src, void* dst,
                  int to_zorder, void* stream) {

@@ -15,9 +15,8 @@
  *  - Layout: every tensor is contiguous [B, H, tokens, D], D innermost.
  *    Q, K, V, O, dO, dQ, dK, dV hold `dtype` elements; pyramids are fp32.
  *  - Index lists I(l): int32 [B, H, N_l, K_l] (K_l = topk_l[l], else topk).
- *    Row q lists the level-l key
- *    tokens kept for level-l query token q, ascending, padded with -1 at the
- *    tail.  Kernels that read index lists use an entry iff it lies in
+ *    Row q lists the level-l key tokens kept for level-l query token q,
+ *    ascending, padded with -1 at the tail.  Kernels that read index lists use an entry iff it lies in
  *    [0, N_l) and is larger than every entry used before it in the row; any
  *    other entry is skipped and reported through `dev_status` (never a fault).
  *  - Memory: the caller allocates and owns every buffer (device memory unless
@@ -29,6 +28,8 @@
  *    on an error nothing is enqueued.
  *  - Device errors: a bit set OR-ed into *dev_status (a device int32 the
  *    caller zeroes and reads after synchronising), if dev_status is not NULL.
+ *  - Versions: llsa_version() changes whenever a struct layout below does;
+ *    bindings that mirror the structs should check it.
  */
 #ifndef LLSA_H_
 #define LLSA_H_

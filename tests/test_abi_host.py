@@ -38,7 +38,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 
 def test_version_and_status_strings(lib):
-    assert llsa.version() == 100
+    assert llsa.version() == llsa.ABI_VERSION == 200
     assert llsa.status_string(llsa.OK) == "ok"
     assert "workspace" in llsa.status_string(llsa.ERR_WORKSPACE)
 
