@@ -5,11 +5,13 @@
 //
 // Pass 1, query-major (bwd_q_mma_kernel): one warp per 16-token query block,
 // 8 sibling blocks per CTA (they share every coarse key).  Selected K/V tiles
-// arrive by 2D TMA loads into a 2-stage per-warp ring; the key list is
-// walked twice:
+// arrive by 2D TMA loads into a 2-stage per-warp ring.  Without the residual
+// of O the key list is walked twice:
 //   sweep 1: S = Q K^T, dP = dO V^T, P = w e^{S - LSE}, Delta_i = sum_j P dP
 //            (from unrounded terms: O is stored rounded);
 //   sweep 2: dS = P (dP - Delta), dQ += dS K.
+// With it (kResid), Delta_i = dO_i . (O_i + R_i) comes first and the list is
+// walked once, as sweep 2.
 // In the sums over queries (dK, dV and the coarse partials) P and dS enter
 // their MMAs as a bf16 hi + lo pair (about 16 mantissa bits): those sums
 // cancel strongly on image-like inputs, and single bf16 rounding left some

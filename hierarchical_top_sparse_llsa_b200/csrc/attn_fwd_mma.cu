@@ -15,7 +15,10 @@
 // The coarse K/V rows (fp32 pyramid) are converted once per CTA to bf16 tiles
 // in shared memory, with ln(w_l) per key folded into the scores.
 // S = Q K^T and O += P V run on m16n8k16 bf16 MMAs with fp32 accumulation;
-// the softmax is online, in base 2, in fp32 registers.
+// the softmax is online, in base 2, in fp32 registers.  When asked for
+// (p.o_res), the epilogue also writes the bf16 rounding residual of O, from
+// which the backward forms Delta without a second walk of the keys; a second
+// instantiation (kSelect) selects I(1) in its prologue.
 
 #include <math.h>
 #include <string.h>
