@@ -26,6 +26,27 @@ def test_algorithmic_work_headline():
     assert abs(work["transpose"]["bytes"] - 4.8e6) < 0.2e6
 
 
+def test_residual_adds_one_tensor_each_way():
+    # the forward writes the bf16 residual of O, the backward reads it
+    w = workloads.WORKLOADS["img256_bf16"]
+    fine = 16 * 65536 * 64 * 2
+    plain, res = bench.algorithmic_work(w), bench.algorithmic_work(w, True)
+    assert res["fwd"]["bytes"] - plain["fwd"]["bytes"] == fine
+    assert res["bwd"]["bytes"] - plain["bwd"]["bytes"] == fine
+    assert res["bwd"]["flops"] == plain["bwd"]["flops"]
+    f32 = workloads.WORKLOADS["tiny_32x32_f32"]
+    assert bench.algorithmic_work(f32, True) == bench.algorithmic_work(f32)  # no residual in fp32
+
+
+def test_gathered_selection_bytes_headline():
+    # per (b, h): level 3 one group of 16 queries scoring all 16 tokens; level 2
+    # 16 groups of 16 queries x 16 * 8 candidates; level 1 256 groups x 128;
+    # plus the Q(l) rows; fp32, D = 64, 16 heads
+    w = workloads.WORKLOADS["img256_bf16"]
+    rows = (1 * 16 + 16) + (16 * 128 + 256) + (256 * 128 + 4096)
+    assert bench.gathered_select_bytes(w) == 16 * rows * 64 * 4
+
+
 def test_launch_count_per_step():
     assert bench.launches_per_step(3) == {"pool": 2, "select": 3, "fwd": 1, "transpose": 4, "bwd": 5}
     assert sum(bench.launches_per_step(2).values()) == 1 + 2 + 1 + 4 + 3
