@@ -15,10 +15,11 @@
 //   scan    one CTA per (level, b, h): the exclusive scan of the totals into
 //           row_ptr, and -1 in the unused tail of col;
 //   fill    one CTA per chunk: the cursors row_ptr[c] + first slot are staged
-//           in shared memory, then one warp walks the chunk's rows in order,
-//           lanes that share a key in one step ranked by __match_any_sync
-//           and advanced by one shared-memory atomic per group, and writes
-//           each query at its key's cursor.
+//           in shared memory, then the chunk's rows go in super-steps of 32
+//           consecutive rows spread over the CTA's warps: each row holding
+//           key c sets its bit in c's row mask (order-free), and after a
+//           barrier each entry's slot is c's cursor plus the number of lower
+//           bits, the highest bit's entry advancing the cursor.
 // Chunks are filled in row order from the slots the prefix gave them, so
 // every key's list comes out ascending and the result is deterministic.
 // Entries are screened with the same used-entry rule as the attention
@@ -34,7 +35,8 @@ constexpr int kCountThreads = 256;
 constexpr int kPrefixThreads = 256;
 constexpr int kPrefixKeys = 4 * kPrefixThreads;  // keys per prefix CTA
 constexpr int kScanThreads = 1024;
-constexpr int kFillThreads = 256;  // all stage the cursors; warp 0 fills
+constexpr int kFillThreads = 256;  // 8 warps: each fills whole rows of a super-step
+constexpr int kSuperRows = 32;     // rows per fill super-step (one bit each in a key's row mask)
 constexpr int kMaxChunks = 128;    // row chunks per (level, b, h); see transpose_chunking
 constexpr int kRangeKeys = 8192;   // keys per shared-memory histogram / cursor range
 constexpr int kBatch = 8;          // row steps whose index loads are in flight together
@@ -200,7 +202,11 @@ tr_scan_kernel(TransposeParams p) {
 
 __global__ void __launch_bounds__(kFillThreads)
 tr_fill_kernel(TransposeParams p) {
-  __shared__ int cur[kRangeKeys];
+  // cur[e]: next free slot of key k0 + e; rowmask[e]: which rows of the
+  // current super-step hold key k0 + e (bit b = row R0 + b)
+  extern __shared__ int fill_smem[];
+  int* cur = fill_smem;
+  unsigned* rowmask = reinterpret_cast<unsigned*>(fill_smem + kRangeKeys);
   const TransposeLevel L = p.lv[level_of(p, blockIdx.x, kChunkGrid)];
   const int local = blockIdx.x - L.cta_begin;
   const int bh = local / L.nchunk, ch = local % L.nchunk;
@@ -212,19 +218,15 @@ tr_fill_kernel(TransposeParams p) {
   int32_t* col = L.col + (size_t)bh * n * K;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const RowLanes rl(K, lane);
+  // a super-step is kSuperRows consecutive rows, rows_per_step per warp
+  const int warp_rows = rl.rows_per_step;
+  const int active_warps = min(kFillThreads / 32, kSuperRows / warp_rows);
+  const int super_rows = active_warps * warp_rows;
 
-  const int step = rl.rows_per_step * kBatch;
-  auto load_batch = [&](int rb, int (&cb)[kBatch]) {
-#pragma unroll
-    for (int i = 0; i < kBatch; ++i) {
-      const int q = rb + i * rl.rows_per_step + rl.sub;
-      cb[i] = (rl.on && q < r1) ? I[(size_t)q * K + rl.slot] : -1;
-    }
-  };
   for (int k0 = 0; k0 < n; k0 += kRangeKeys) {
     const int len = min(n, k0 + kRangeKeys) - k0;
     // cursors: the key's first slot plus this chunk's offset in its list,
-    // 8 pairs of loads in flight per thread
+    // 8 pairs of loads in flight per thread; masks cleared
     for (int e0 = threadIdx.x; e0 < len; e0 += 8 * kFillThreads) {
       int t[8];
 #pragma unroll
@@ -235,54 +237,41 @@ tr_fill_kernel(TransposeParams p) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         const int e = e0 + i * kFillThreads;
-        if (e < len) cur[e] = t[i];
+        if (e < len) {
+          cur[e] = t[i];
+          rowmask[e] = 0u;
+        }
       }
     }
     __syncthreads();
-    if (warp == 0) {
+    for (int R0 = r0; R0 < r1; R0 += super_rows) {
+      // this lane's entry: row R0 + b of the super-step
+      const int b = warp * warp_rows + rl.sub;
+      const int q = R0 + b;
+      const bool row_on = warp < active_warps && rl.on && q < r1;
+      const int c = row_on ? I[(size_t)q * K + rl.slot] : -1;
       int dummy = 0;
-      int cb[kBatch], nb[kBatch];
-      load_batch(r0, cb);
-      for (int rb = r0; rb < r1; rb += step) {
-        load_batch(rb + step, nb);  // the next batch's loads overlap this batch
-        // the steps' screening and ranking are independent of one another
-        int key[kBatch], rank[kBatch];
-        unsigned peers[kBatch];
-#pragma unroll
-        for (int i = 0; i < kBatch; ++i) {
-          const int q = rb + i * rl.rows_per_step + rl.sub;
-          const int c = cb[i];
-          const bool u = warp_row_used(c, rl.slot, n, rl.on && q < r1, dummy, K);
-          key[i] = (u && c >= k0 && c < k0 + len) ? c - k0 : -1 - lane;  // -1 - lane matches nobody
-          if (rl.rows_per_step == 1) {
-            // one row per step: its used entries are distinct keys
-            peers[i] = 1u << lane;
-            rank[i] = 0;
-          } else {
-            peers[i] = __match_any_sync(0xffffffffu, key[i]);
-            rank[i] = __popc(peers[i] & ((1u << lane) - 1u));  // lower lanes hold lower rows
-          }
-        }
-        // The cursor updates run in step order: the highest lane of each group
-        // of lanes sharing a key takes the group's slots with one shared-memory
-        // atomic (one warp instruction per step, so same-key atomics of
-        // consecutive steps are applied in step order) and hands the base to
-        // its group by a shuffle.  No warp barrier is needed between steps, so
-        // none waits for the scattered stores into col.
-#pragma unroll
-        for (int i = 0; i < kBatch; ++i) {
-          const int q = rb + i * rl.rows_per_step + rl.sub;
-          const int leader = 31 - __clz(peers[i]);
-          int base = 0;
-          if (key[i] >= 0 && lane == leader) base = atomicAdd(&cur[key[i]], __popc(peers[i]));
-          if (rl.rows_per_step > 1) base = __shfl_sync(0xffffffffu, base, leader);
-          if (key[i] >= 0) col[base + rank[i]] = q;
-        }
-#pragma unroll
-        for (int i = 0; i < kBatch; ++i) cb[i] = nb[i];
+      const bool u = warp_row_used(c, rl.slot, n, row_on, dummy, K);
+      const int key = (u && c >= k0 && c < k0 + len) ? c - k0 : -1;
+      // 1. every row that holds a key marks its bit (order-free)
+      if (key >= 0) atomicOr(&rowmask[key], 1u << b);
+      __syncthreads();
+      // 2. slot = cursor + the rows before this one in the super-step that
+      //    hold the key; the last such row advances the cursor after all reads
+      bool last = false;
+      unsigned m = 0u;
+      if (key >= 0) {
+        m = rowmask[key];
+        col[cur[key] + __popc(m & ((1u << b) - 1u))] = q;
+        last = (31 - __clz(m)) == b;
       }
+      __syncthreads();
+      if (last) {
+        cur[key] += __popc(m);
+        rowmask[key] = 0u;
+      }
+      __syncthreads();
     }
-    __syncthreads();  // cur is restaged for the next key range
   }
 }
 
@@ -314,7 +303,10 @@ cudaError_t launch_transpose(const TransposeParams& p, cudaStream_t s) {
   tr_scan_kernel<<<scans, kScanThreads, 0, s>>>(p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  tr_fill_kernel<<<chunks, kFillThreads, 0, s>>>(p);
+  const size_t fill_smem = (size_t)kRangeKeys * (sizeof(int) + sizeof(unsigned));
+  e = cudaFuncSetAttribute(tr_fill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)fill_smem);
+  if (e != cudaSuccess) return e;
+  tr_fill_kernel<<<chunks, kFillThreads, fill_smem, s>>>(p);
   return cudaGetLastError();
 }
 
