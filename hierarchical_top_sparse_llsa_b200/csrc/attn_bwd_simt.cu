@@ -46,7 +46,6 @@ bwd_query_simt_kernel(AttnParams p, int G) {
   const int bh = blockIdx.y;
   const int tid = threadIdx.x;
   const int i = tid >> 4, sub = tid & 15;
-  const int K = p.K;
   const int NG = p.N >> 7;  // partial groups of 8 query blocks per (b, h)
   const T* Q = static_cast<const T*>(p.q);
   const T* Kf = static_cast<const T*>(p.k);

@@ -244,12 +244,19 @@ tr_fill_kernel(TransposeParams p) {
       }
     }
     __syncthreads();
+    // this lane's entry is row R0 + b of each super-step; the next
+    // super-step's entry is loaded while the current one is placed
+    const int b = warp * warp_rows + rl.sub;
+    auto entry = [&](int R0) {
+      const int q = R0 + b;
+      return (warp < active_warps && rl.on && q < r1) ? I[(size_t)q * K + rl.slot] : -1;
+    };
+    int c_next = entry(r0);
     for (int R0 = r0; R0 < r1; R0 += super_rows) {
-      // this lane's entry: row R0 + b of the super-step
-      const int b = warp * warp_rows + rl.sub;
       const int q = R0 + b;
       const bool row_on = warp < active_warps && rl.on && q < r1;
-      const int c = row_on ? I[(size_t)q * K + rl.slot] : -1;
+      const int c = c_next;
+      if (R0 + super_rows < r1) c_next = entry(R0 + super_rows);
       int dummy = 0;
       const bool u = warp_row_used(c, rl.slot, n, row_on, dummy, K);
       const int key = (u && c >= k0 && c < k0 + len) ? c - k0 : -1;
