@@ -6,10 +6,15 @@
     python bench.py --impl reference ...   (the CPU oracle, timed the same way)
 
 One step is one pass of the whole path over one batch of seeded synthetic
-input already resident in device memory.  Every GPU runs its own copy of the
-workload (heads and batches are independent, so the path shards with no
+input already resident in device memory, replayed as one CUDA graph; the
+forward and backward go through the residual calls (llsa_attn_fwd_res /
+llsa_attn_bwd_res) unless --no-residual.  Every GPU runs its own copy of
+the workload (heads and batches are independent, so the path shards with no
 collective): per-GPU work is fixed as N grows, i.e. weak scaling.  Rank 0
-prints one JSON line.
+prints one JSON line: the step rate, per-stage times against their
+rooflines, the end-to-end rate with host copies (pipelined over steps), the
+oracle on the host cores, a dense-attention reference, the index transpose
+timed back to back and the Z-order permutation's bandwidth.
 """
 
 from __future__ import annotations
@@ -18,15 +23,12 @@ import argparse
 import hashlib
 import datetime
 import json
-import math
 import os
 import re
 import statistics
 import subprocess
 import sys
 import time
-
-import numpy as np
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
