@@ -1,6 +1,6 @@
 """Build libllsa.so (sm_100a) in-tree with nvcc.
 
-    python -m hierarchical_top_sparse_llsa_b200.build [--debug]
+    python -m hierarchical_top_sparse_llsa_b200.build [-v]      (-v: ptxas resource usage)
 
 The shared library is written next to this file, so it travels with the
 source tree and the Python binding finds it without any install step.
