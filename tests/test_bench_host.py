@@ -111,3 +111,25 @@ def test_max_over_ranks_two_gloo_ranks():
             p.join(100)
         assert all(p.exitcode == 0 for p in procs)
         assert out[0] == [2.0, 10.0] and out[1] == [2.0, 10.0]
+
+
+@pytest.mark.parametrize("rank", [0, 1])
+def test_reference_arm_under_two_ranks(rank):
+    # launched as one of two ranks: rank 0 alone times the oracle and prints
+    # the line; the other rank exits 0 without work
+    import json
+    import subprocess
+    import sys
+
+    env = dict(os.environ, RANK=str(rank), WORLD_SIZE="2", LOCAL_RANK=str(rank))
+    out = subprocess.run([sys.executable, os.path.join(os.path.dirname(bench.__file__), "bench.py"),
+                          "--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "0",
+                          "--workload", "tiny_32x32_f32"], env=env, capture_output=True, text=True, timeout=600)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.strip()]
+    if rank == 0:
+        rec = json.loads(lines[-1])
+        assert rec["impl"] == "reference" and rec["n_gpus"] == 2 and rec["value"] > 0
+        assert rec["e2e"]["h2d_bytes_per_step"] == 0 and rec["cpu_baseline"]["kind"] == "oracle"
+    else:
+        assert lines == []
