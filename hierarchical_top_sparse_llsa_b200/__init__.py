@@ -29,6 +29,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_LAUNCH, ERR_WORKSPACE = 0, 1, 2, 3, 4
 DEV_BAD_INDEX, DEV_NONCANONICAL, DEV_TIMEOUT = 1, 2, 4
 FLAG_FWD_TCGEN05 = 1
 FLAG_BWD_TCGEN05 = 2
+FLAG_FWD_MMA_SYNC = 4
 NOALLOC_SCRATCH_BYTES = 16 << 20
 
 EXPORTED = (
@@ -44,6 +45,7 @@ EXPORTED = (
     "llsa_attn_bwd",
     "llsa_attn_bwd_noalloc",
     "llsa_reorder",
+    "llsa_selftest_wait_timeout",
     "llsa_status_string",
     "llsa_version",
 )
@@ -118,6 +120,7 @@ def lib() -> ctypes.CDLL:
                                                      P(LlsaIndices), P(LlsaCsr), vp, vp, vp, vp, vp]),
             "llsa_reorder": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                             ctypes.c_int, vp, vp, ctypes.c_int, vp]),
+            "llsa_selftest_wait_timeout": (ctypes.c_int, [vp, ctypes.c_uint, vp]),
             "llsa_status_string": (ctypes.c_char_p, [ctypes.c_int]),
             "llsa_version": (ctypes.c_int, []),
         }
@@ -237,6 +240,13 @@ def llsa_attn_bwd_noalloc(desc, q, k, v, pyramid, o, lse, dout, indices, csr, dq
     st = lib().llsa_attn_bwd_noalloc(ctypes.byref(desc), q, k, v, ctypes.byref(pyramid), o, lse, dout,
                                      ctypes.byref(indices), ctypes.byref(csr), dq, dk, dv, dev_status,
                                      stream)
+    return _check(st) if check else st
+
+
+def llsa_selftest_wait_timeout(dev_status, limit_us, stream=0, check=True):
+    """One launch that drives the kernels' bounded mbarrier wait to expiry
+    (nothing arrives): LLSA_DEV_TIMEOUT is OR-ed into *dev_status."""
+    st = lib().llsa_selftest_wait_timeout(dev_status, limit_us, stream)
     return _check(st) if check else st
 
 

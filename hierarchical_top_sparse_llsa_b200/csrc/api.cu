@@ -16,18 +16,13 @@ cudaError_t launch_attn_fwd_mma(const AttnParams& p, const CUtensorMap* maps, cu
 cudaError_t launch_attn_fwd_mma_select(const AttnParams& p, const SelectParams& sp, const CUtensorMap* maps,
                                        cudaStream_t s);
 cudaError_t launch_attn_fwd_tc(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s);
+size_t attn_fwd_tc_smem(const AttnParams& p);
 cudaError_t launch_attn_bwd_mma(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s, bool tc_kv);
 }  // namespace llsa
 
 using namespace llsa;
 
 namespace {
-
-// The tcgen05 forward (attn_fwd_tc.cu) is the bf16 D = 64 default only when
-// it is the faster of the two; LLSA_FLAG_FWD_TCGEN05 selects it explicitly.
-constexpr bool kUseTcForward = false;
-// Likewise for the key-major backward pass; LLSA_FLAG_BWD_TCGEN05 selects it.
-constexpr bool kUseTcBackward = false;
 
 // K_l, the width of I(l): topk_l[l], or topk where that is 0.
 inline int k_level(const llsa_desc* d, int l) { return d->topk_l[l] > 0 ? d->topk_l[l] : d->topk; }
@@ -36,7 +31,9 @@ inline int check_desc(const llsa_desc* d) {
   if (d == nullptr) return LLSA_ERR_INVALID_ARG;
   if (d->B < 1 || d->H < 1 || d->N < kBlock || d->D < 1 || d->L < 1 || d->topk < 1)
     return LLSA_ERR_INVALID_ARG;
-  if ((d->flags & ~(LLSA_FLAG_FWD_TCGEN05 | LLSA_FLAG_BWD_TCGEN05)) != 0) return LLSA_ERR_INVALID_ARG;
+  if ((d->flags & ~(LLSA_FLAG_FWD_TCGEN05 | LLSA_FLAG_BWD_TCGEN05 | LLSA_FLAG_FWD_MMA_SYNC)) != 0)
+    return LLSA_ERR_INVALID_ARG;
+  if ((d->flags & LLSA_FLAG_FWD_TCGEN05) && (d->flags & LLSA_FLAG_FWD_MMA_SYNC)) return LLSA_ERR_INVALID_ARG;
   if (d->dtype != LLSA_F32 && d->dtype != LLSA_BF16) return LLSA_ERR_INVALID_ARG;
   if (d->D != 64 && d->D != 128) return LLSA_ERR_UNSUPPORTED;
   if (d->L > kMaxL || d->topk > kMaxK) return LLSA_ERR_UNSUPPORTED;
@@ -141,15 +138,15 @@ EncodeTiledFn encode_tiled() {
   return fn;
 }
 
-// A bf16 [rows, D] row-major tensor seen by TMA as tiles of 16 rows x 64
-// columns (128 bytes) with 128-byte swizzle.
-int make_row_tile_map(CUtensorMap* map, const void* base, uint64_t rows, int D) {
+// A bf16 [rows, D] row-major tensor seen by TMA as tiles of box_rows rows x
+// 64 columns (128 bytes) with 128-byte swizzle.
+int make_row_tile_map(CUtensorMap* map, const void* base, uint64_t rows, int D, int box_rows = 16) {
   EncodeTiledFn fn = encode_tiled();
   if (fn == nullptr) return LLSA_ERR_LAUNCH;
   if ((reinterpret_cast<uintptr_t>(base) & 15) != 0) return LLSA_ERR_INVALID_ARG;
   const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  const cuuint32_t box[2] = {64, 16};
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   const cuuint32_t estride[2] = {1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                         strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -222,13 +219,17 @@ enum class FwdPath { kSimt, kTc, kMma };
 
 struct FwdPlan {
   AttnParams p;
-  CUtensorMap maps[3];
+  CUtensorMap maps[5];  // Q, K, V loads; O and its residual stores (tcgen05 path)
   FwdPath path;
 };
 
+// Shared memory per CTA that kernels may use (B200: 227 KB).
+constexpr size_t kMaxSmemPerCta = 227 * 1024;
+
 // Every check of the forward (and its tensor maps), before anything launches.
+// o_res: the residual of O to write (bf16 only), or NULL.
 int plan_fwd(const llsa_desc* desc, const void* q, const void* k, const void* v, const llsa_pyramid* pyr,
-             const llsa_indices* idx, void* o, float* lse, int32_t* dev_status, FwdPlan& f) {
+             const llsa_indices* idx, void* o, void* o_res, float* lse, int32_t* dev_status, FwdPlan& f) {
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || lse == nullptr ||
       idx == nullptr || pyr == nullptr)
     return LLSA_ERR_INVALID_ARG;
@@ -250,8 +251,17 @@ int plan_fwd(const llsa_desc* desc, const void* q, const void* k, const void* v,
     const int st = make_row_tile_map(&f.maps[i], srcs[i], rows, desc->D);
     if (st != LLSA_OK) return st;
   }
-  const bool use_tc = kUseTcForward || (desc->flags & LLSA_FLAG_FWD_TCGEN05) != 0;
-  f.path = (use_tc && desc->D == 64) ? FwdPath::kTc : FwdPath::kMma;  // tcgen05: MMAs into tensor memory
+  // tcgen05 (tensor-memory accumulators) unless the warp-MMA kernel is asked
+  // for, or the coarse keys need more shared memory than a CTA has
+  memset(&f.maps[3], 0, 2 * sizeof(CUtensorMap));
+  f.path = FwdPath::kMma;
+  if ((desc->flags & LLSA_FLAG_FWD_MMA_SYNC) == 0 && attn_fwd_tc_smem(f.p) <= kMaxSmemPerCta) {
+    f.path = FwdPath::kTc;
+    int st = make_row_tile_map(&f.maps[3], o, rows, desc->D, 128);
+    if (st == LLSA_OK && o_res != nullptr) st = make_row_tile_map(&f.maps[4], o_res, rows, desc->D, 128);
+    if (st != LLSA_OK) return st;
+  }
+  f.p.o_res = o_res;
   return LLSA_OK;
 }
 
@@ -349,7 +359,7 @@ int llsa_attn_fwd(const llsa_desc* desc, const void* q, const void* k, const voi
   int st = check_desc(desc);
   if (st != LLSA_OK) return st;
   FwdPlan f;
-  st = plan_fwd(desc, q, k, v, pyr, idx, o, lse, dev_status, f);
+  st = plan_fwd(desc, q, k, v, pyr, idx, o, nullptr, lse, dev_status, f);
   if (st != LLSA_OK) return st;
   return launch_fwd(f, (cudaStream_t)stream);
 }
@@ -362,7 +372,7 @@ int llsa_select_attn_fwd(const llsa_desc* desc, const void* q, const void* k, co
   st = check_select_args(desc, pyr, idx);
   if (st != LLSA_OK) return st;
   FwdPlan f;
-  st = plan_fwd(desc, q, k, v, pyr, idx, o, lse, dev_status, f);
+  st = plan_fwd(desc, q, k, v, pyr, idx, o, nullptr, lse, dev_status, f);
   if (st != LLSA_OK) return st;
   const cudaStream_t s = (cudaStream_t)stream;
   const int BH = desc->B * desc->H;
@@ -447,13 +457,10 @@ int llsa_attn_fwd_res(const llsa_desc* desc, const void* q, const void* k, const
   if (st != LLSA_OK) return st;
   if (desc->dtype == LLSA_BF16) {  // fp32: O is not rounded, o_res is not used
     if (o_res == nullptr || ((uintptr_t)o_res & 15) != 0) return LLSA_ERR_INVALID_ARG;
-    if (kUseTcForward || (desc->flags & LLSA_FLAG_FWD_TCGEN05) != 0)
-      return LLSA_ERR_UNSUPPORTED;  // the residual comes from the warp-MMA kernel
   }
   FwdPlan f;
-  st = plan_fwd(desc, q, k, v, pyr, idx, o, lse, dev_status, f);
+  st = plan_fwd(desc, q, k, v, pyr, idx, o, desc->dtype == LLSA_BF16 ? o_res : nullptr, lse, dev_status, f);
   if (st != LLSA_OK) return st;
-  if (f.path == FwdPath::kMma) f.p.o_res = o_res;
   return launch_fwd(f, (cudaStream_t)stream);
 }
 
@@ -512,7 +519,7 @@ int attn_bwd_impl(const llsa_desc* desc, const void* q, const void* k, const voi
     st = make_row_tile_map(&maps[i], srcs[i], rows, desc->D);
     if (st != LLSA_OK) return st;
   }
-  const bool tc_kv = kUseTcBackward || (desc->flags & LLSA_FLAG_BWD_TCGEN05) != 0;
+  const bool tc_kv = (desc->flags & LLSA_FLAG_BWD_TCGEN05) != 0;
   return launch_status(launch_attn_bwd_mma(p, maps, (cudaStream_t)stream, tc_kv));
 }
 

@@ -13,14 +13,19 @@
 // (16 MiB).  Every GPU that loads this library holds it until the process
 // exits.  Host code cannot use the array's name as a device address (in host
 // code it names a host-side stand-in), so its device address is looked up
-// with cudaGetSymbolAddress once per device, with that device current, on
-// the first call made on that device, and cached.
+// with cudaGetSymbolAddress, with the device current, on the first call made
+// on that device, and cached together with the CUDA context it belongs to.
+// A later call under another context of the same device (after
+// cudaDeviceReset, say, which reloads the library's module at a possibly
+// different address) looks the address up again.
 //
 // All calls share the one array and it keeps whatever the last call wrote.
 // Nothing in it has to start at zero: the backward kernels zero their own
 // partial sums and write every other scratch word before reading it.  Two
 // calls whose work overlaps on the GPU (for instance on two streams) race
 // on the array and give wrong results; serialise them.
+
+#include <cuda.h>
 
 #include <mutex>
 
@@ -32,21 +37,48 @@ constexpr size_t kScratchBytes = LLSA_NOALLOC_SCRATCH_BYTES;
 static __device__ __align__(256) unsigned char g_bwd_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
+struct CachedAddress {
+  CUcontext ctx;
+  void* addr;
+};
 std::mutex g_mutex;
-void* g_scratch_addr[kMaxDevices] = {};
+CachedAddress g_scratch[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device (set up once).
+// cuCtxGetCurrent from the driver (no link-time libcuda), fetched once.
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+CtxGetCurrentFn ctx_get_current() {
+  static CtxGetCurrentFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(f);
+  });
+  return fn;
+}
+
+// Device address of the scratch array on the current device, looked up on
+// the first call under each context of the device.
 int scratch_on_current_device(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LLSA_ERR_LAUNCH;
+  CtxGetCurrentFn get_ctx = ctx_get_current();
+  if (get_ctx == nullptr) return LLSA_ERR_LAUNCH;
   std::lock_guard<std::mutex> lock(g_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
-    void* p = nullptr;
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) return LLSA_ERR_LAUNCH;
+  CachedAddress& c = g_scratch[dev];
+  if (ctx == nullptr || ctx != c.ctx || c.addr == nullptr) {
+    void* p = nullptr;  // the lookup also makes the device's context current
     const cudaError_t e = cudaGetSymbolAddress(&p, g_bwd_scratch);
     if (e != cudaSuccess || p == nullptr) return LLSA_ERR_LAUNCH;
-    g_scratch_addr[dev] = p;
+    if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return LLSA_ERR_LAUNCH;
+    c.ctx = ctx;
+    c.addr = p;
   }
-  *out = g_scratch_addr[dev];
+  *out = c.addr;
   return LLSA_OK;
 }
 

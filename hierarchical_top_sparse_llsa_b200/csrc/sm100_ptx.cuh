@@ -46,14 +46,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait for phase `parity` of a barrier, giving up after a bounded number of
-// polls (each poll may itself suspend for a short hardware-defined time).
-// Returns false on time-out; the caller reports LLSA_DEV_TIMEOUT.
-constexpr uint32_t kMaxPolls = 1u << 24;
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
-  for (uint32_t i = 0; i < kMaxPolls; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
-  return false;
+// Nanoseconds of the GPU's global timer.
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for phase `parity` of a barrier for at most `limit_ns` nanoseconds of
+// the global timer (checked every 32 polls; a poll may itself suspend for a
+// short hardware-defined time).  Returns false on time-out; the caller then
+// reports LLSA_DEV_TIMEOUT.  The default limit, 1 s, is far above any wait of
+// a correct launch (the longest kernel of the path runs for about a
+// millisecond) and short enough that a lost arrival ends the launch instead
+// of holding the GPU.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  uint64_t limit_ns = kWaitLimitNs) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > limit_ns) return false;
+  }
 }
 
 // Order this thread's earlier generic-proxy shared-memory accesses before
@@ -71,6 +88,23 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
       : "memory");
 }
+
+// 2D TMA tile store from shared memory (bulk-group completion): the tile at
+// `src` (laid out as the tensor map's box, with its swizzle) goes to
+// coordinates (x, y).  The issuing thread commits and waits for the group.
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, int x, int y, uint32_t src) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(src)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until every committed bulk store of this thread has finished reading
+// shared memory (`read`) or has completed
+__device__ __forceinline__ void bulk_wait_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 // 1D bulk copy (no tensor map) of `bytes` (a multiple of 16, both addresses
 // 16-byte aligned) into shared memory, completing on `bar`.  No multicast.

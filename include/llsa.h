@@ -65,14 +65,22 @@ enum {
 
 /* descriptor flags */
 enum {
-  /* bf16, D = 64: run llsa_attn_fwd on the tcgen05 kernel (tensor-memory
-   * accumulators, 8 sibling query blocks per 128-row MMA) instead of the
-   * warp-MMA kernel.  Both compute the same result within bf16 rounding. */
+  /* bf16: the forward on the tcgen05 kernel (tensor-memory accumulators, 8
+   * sibling query blocks per 128-row MMA).  This is the default for bf16; the
+   * flag states it explicitly and excludes LLSA_FLAG_FWD_MMA_SYNC. */
   LLSA_FLAG_FWD_TCGEN05 = 1,
   /* bf16, D = 64: run the key-major pass of llsa_attn_bwd (dK, dV) on the
    * tcgen05 kernel (8 query blocks of a key block per 128-row MMA, dK and dV
    * accumulated in tensor memory) instead of the warp-MMA kernel. */
-  LLSA_FLAG_BWD_TCGEN05 = 2
+  LLSA_FLAG_BWD_TCGEN05 = 2,
+  /* bf16: run the forward (llsa_attn_fwd, llsa_attn_fwd_res and the forward of
+   * llsa_select_attn_fwd) on the warp-level mma.sync kernel (one warp per 4
+   * query blocks, registers as accumulators) instead of the tcgen05 kernel,
+   * for comparison.  Both compute the same result within bf16 rounding.  The
+   * library also takes this kernel by itself when the coarse keys of one CTA
+   * need more shared memory than the tcgen05 kernel has (the sum of K_l over
+   * levels 2..Lc above 128 at D = 128). */
+  LLSA_FLAG_FWD_MMA_SYNC = 4
 };
 
 /* device status bits (OR-ed into *dev_status) */
@@ -188,9 +196,10 @@ LLSA_API int llsa_attn_fwd(const llsa_desc* desc, const void* q, const void* k, 
  *   Arguments as the two calls take them: pyr holds q[l], k[l] for l = 1..L
  *   and k[l], v[l] for l = 2..Lc; idx: I(1..L), all written (as llsa_select
  *   writes them; the backward needs them).  Results are identical to the two
- *   calls made one after the other.  The bf16 warp-MMA forward fuses; with
- *   fp32 or LLSA_FLAG_FWD_TCGEN05 the level-1 selection runs as its own
- *   launch before the forward.
+ *   calls made one after the other.  The fusion is done by the warp-MMA
+ *   forward (LLSA_FLAG_FWD_MMA_SYNC); on the tcgen05 forward (the bf16
+ *   default) and in fp32 the level-1 selection runs as its own launch before
+ *   the forward.
  */
 LLSA_API int llsa_select_attn_fwd(const llsa_desc* desc, const void* q, const void* k, const void* v,
                                   const llsa_pyramid* pyr, const llsa_indices* idx, void* o, float* lse,
@@ -205,7 +214,6 @@ LLSA_API int llsa_select_attn_fwd(const llsa_desc* desc, const void* q, const vo
  *   fp32 output before rounding; o + o_res then holds O to about 16 mantissa
  *   bits.  o and lse are identical to llsa_attn_fwd's.
  *   dtype LLSA_F32: O is stored unrounded, o_res is not used (may be NULL).
- *   LLSA_FLAG_FWD_TCGEN05 with bf16 gives LLSA_ERR_UNSUPPORTED.
  */
 LLSA_API int llsa_attn_fwd_res(const llsa_desc* desc, const void* q, const void* k, const void* v,
                                const llsa_pyramid* pyr, const llsa_indices* idx, void* o, void* o_res,
@@ -296,8 +304,10 @@ LLSA_API int llsa_attn_bwd_res(const llsa_desc* desc, const void* q, const void*
  *     LLSA_NOALLOC_SCRATCH_BYTES the call returns LLSA_ERR_WORKSPACE and
  *     enqueues nothing (use llsa_attn_bwd with your own workspace instead).
  *   - Set-up: the first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current) and caches it; make
- *     that first call before any stream capture.
+ *     (cudaGetSymbolAddress, with that device current) and caches it with
+ *     the device's CUDA context; make that first call before any stream
+ *     capture.  The first call under a new context of the device (after
+ *     cudaDeviceReset, for instance) looks it up again.
  *   - Sharing: every call uses the same array, which keeps the last call's
  *     contents (nothing in it needs to start at zero).  Calls whose work
  *     overlaps on the GPU race on it and give wrong results: serialise them.
@@ -324,6 +334,21 @@ LLSA_API int llsa_attn_bwd_noalloc(const llsa_desc* desc, const void* q, const v
  */
 LLSA_API int llsa_reorder(int B, int H, int img_h, int img_w, int D, int dtype, const void* src, void* dst,
                           int to_zorder, void* stream);
+
+/*
+ * llsa_selftest_wait_timeout - a check of the kernels' bounded waits.
+ *   The paper has no counterpart: this is a test hook of this library.  The
+ *   attention kernels wait on mbarriers for their copies and tensor-core
+ *   results; every such wait gives up after a time limit (1 s of the GPU's
+ *   global timer), reports LLSA_DEV_TIMEOUT in *dev_status and lets the
+ *   kernel return, so a lost arrival never holds the GPU.  This call
+ *   launches one kernel that runs the same wait on a barrier nothing arrives
+ *   on, with a limit of limit_us microseconds, so a caller can see the
+ *   time-out reported without any fault.
+ *   dev_status: device int32 (required); LLSA_DEV_TIMEOUT is OR-ed into it.
+ *   limit_us: 1 .. 2,000,000 (else LLSA_ERR_INVALID_ARG, nothing enqueued).
+ */
+LLSA_API int llsa_selftest_wait_timeout(int32_t* dev_status, unsigned limit_us, void* stream);
 
 /* Static text for a host status code. */
 LLSA_API const char* llsa_status_string(int status);

@@ -57,7 +57,8 @@ def _desc(**kw):
     (dict(topk=0), llsa.ERR_INVALID_ARG),
     (dict(dtype=5), llsa.ERR_INVALID_ARG),
     (dict(B=0), llsa.ERR_INVALID_ARG),
-    (dict(flags=4), llsa.ERR_INVALID_ARG),
+    (dict(flags=8), llsa.ERR_INVALID_ARG),  # an unknown flag bit
+    (dict(flags=llsa.FLAG_FWD_TCGEN05 | llsa.FLAG_FWD_MMA_SYNC), llsa.ERR_INVALID_ARG),  # two forwards
 ])
 def test_bad_descriptors_are_rejected_before_launch(lib, kw, status):
     d = _desc(**kw)
@@ -240,3 +241,10 @@ def test_residual_calls_check_arguments(lib):
     ws = llsa.llsa_bwd_workspace_bytes(d)
     assert llsa.llsa_attn_bwd_res(d, 256, 256, 256, pyr, 256, 264, 256, 256, ind, csr, 256, 256, 256,
                                   256, ws - 1, check=False) == llsa.ERR_WORKSPACE
+
+
+def test_wait_timeout_selftest_checks_arguments(lib):
+    # host checks come before any launch: nothing reaches a device here
+    assert llsa.llsa_selftest_wait_timeout(None, 10, check=False) == llsa.ERR_INVALID_ARG
+    assert llsa.llsa_selftest_wait_timeout(256, 0, check=False) == llsa.ERR_INVALID_ARG
+    assert llsa.llsa_selftest_wait_timeout(256, 2000001, check=False) == llsa.ERR_INVALID_ARG

@@ -167,11 +167,12 @@ def test_runs_are_bitwise_deterministic():
     ("img128_bf16", [3]),
     ("img256_bf16", [7]),
 ])
-def test_tcgen05_forward(name, heads):
-    # the tcgen05 forward kernel, selected by LLSA_FLAG_FWD_TCGEN05
+def test_mma_sync_forward(name, heads):
+    # the warp-level mma.sync forward kernel, selected by LLSA_FLAG_FWD_MMA_SYNC
+    # (the default bf16 forward is the tcgen05 kernel, covered by every other test)
     w = workloads.WORKLOADS[name]
     x = workloads.make_inputs(w)
-    g = run_gpu(w.B, w.H, w.N, w.D, w.L, w.topk, w.dtype, x, bwd=False, flags=llsa.FLAG_FWD_TCGEN05)
+    g = run_gpu(w.B, w.H, w.N, w.D, w.L, w.topk, w.dtype, x, bwd=False, flags=llsa.FLAG_FWD_MMA_SYNC)
     assert g["status"] == 0
     hs = slice(None) if heads is None else heads
     xs = x if heads is None else {k: np.ascontiguousarray(v[:, heads]) for k, v in x.items()}
@@ -179,7 +180,40 @@ def test_tcgen05_forward(name, heads):
     _compare(w, g, r, hs, False)
 
 
-@pytest.mark.parametrize("flags", [0, llsa.FLAG_FWD_TCGEN05])
+@pytest.mark.parametrize("N,D", [(192, 64), (3 * 256 + 64, 128)])
+def test_tcgen05_forward_partial_cta(N, D):
+    # a CTA owns 8 query blocks; here the last one owns fewer (12 and 52
+    # blocks), so its rows are stored by the threads rather than by TMA
+    x = _small(41, 1, 2, N, D)
+    g = run_gpu(1, 2, N, D, 1, 4, "bf16", x, bwd=False, resid=True)
+    r = run_oracle(x, 1, 4, bwd=False)
+    assert g["status"] == 0
+    assert_close(g["O"], r["O"], "bf16", "O")
+    assert_close(g["LSE"], r["LSE"], "bf16", "LSE")
+    # o + residual carries O to far below bf16 rounding
+    err = np.abs(g["O"] + g["O_res"] - r["O"]).max()
+    assert err < 2e-3 * np.abs(r["O"]).max(), err
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_tcgen05_forward_rising_maximum(D):
+    # keys whose magnitude grows with their block index, every block of the
+    # single level kept (K = 32 of 32): each row's maximum rises chunk after
+    # chunk by far more than the 2^8 the forward lets its reference lag, so
+    # O and l are rescaled in tensor memory repeatedly
+    B, H, N, L, K = 1, 2, 512, 1, 32
+    x = _small(42, B, H, N, D)
+    scale = np.repeat(np.linspace(0.2, 6.0, N // 16), 16).astype(np.float32)
+    x["k"] = workloads.round_to_bf16(x["k"] * scale[None, None, :, None])
+    g = run_gpu(B, H, N, D, L, K, "bf16", x, bwd=False)
+    r = run_oracle(x, L, K, bwd=False)
+    assert g["status"] == 0
+    assert np.all(g["idx"][1] >= 0)
+    assert_close(g["O"], r["O"], "bf16", "O")
+    assert_close(g["LSE"], r["LSE"], "bf16", "LSE")
+
+
+@pytest.mark.parametrize("flags", [0, llsa.FLAG_FWD_MMA_SYNC])
 def test_forward_external_indices_and_weights(flags):
     B, H, N, D, L, K = 1, 2, 4096, 64, 3, 6
     x = _small(27, B, H, N, D)
@@ -245,6 +279,7 @@ def test_tcgen05_backward_external_indices_and_long_rows():
     (-1, 0),
     (1, 0),
     (1, llsa.FLAG_FWD_TCGEN05 | llsa.FLAG_BWD_TCGEN05),
+    (1, llsa.FLAG_FWD_MMA_SYNC),
     (2, 0),
 ])
 def test_enrichment_depth(enrich, flags):
@@ -277,6 +312,7 @@ def test_enrichment_depth(enrich, flags):
     ("bf16", 0, {1: 4, 2: 16, 3: 1}),
     ("bf16", 0, {1: 20, 2: 1, 3: 1}),   # 16 level-1 candidates: four pads per row
     ("bf16", llsa.FLAG_FWD_TCGEN05 | llsa.FLAG_BWD_TCGEN05, {1: 12, 2: 4, 3: 2}),
+    ("bf16", llsa.FLAG_FWD_MMA_SYNC, {1: 12, 2: 4, 3: 2}),
     ("f32", 0, {1: 6, 2: 3, 3: 2}),
 ])
 def test_topk_per_level(dtype, flags, kl):
