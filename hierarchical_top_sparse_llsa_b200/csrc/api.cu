@@ -138,15 +138,15 @@ EncodeTiledFn encode_tiled() {
   return fn;
 }
 
-// A bf16 [rows, D] row-major tensor seen by TMA as tiles of box_rows rows x
-// 64 columns (128 bytes) with 128-byte swizzle.
-int make_row_tile_map(CUtensorMap* map, const void* base, uint64_t rows, int D, int box_rows = 16) {
+// A bf16 [rows, D] row-major tensor seen by TMA as tiles of 16 rows x 64
+// columns (128 bytes) with 128-byte swizzle.
+int make_row_tile_map(CUtensorMap* map, const void* base, uint64_t rows, int D) {
   EncodeTiledFn fn = encode_tiled();
   if (fn == nullptr) return LLSA_ERR_LAUNCH;
   if ((reinterpret_cast<uintptr_t>(base) & 15) != 0) return LLSA_ERR_INVALID_ARG;
   const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  const cuuint32_t box[2] = {64, 16};
   const cuuint32_t estride[2] = {1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                         strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -219,7 +219,7 @@ enum class FwdPath { kSimt, kTc, kMma };
 
 struct FwdPlan {
   AttnParams p;
-  CUtensorMap maps[5];  // Q, K, V loads; O and its residual stores (tcgen05 path)
+  CUtensorMap maps[3];  // Q, K, V
   FwdPath path;
 };
 
@@ -253,14 +253,8 @@ int plan_fwd(const llsa_desc* desc, const void* q, const void* k, const void* v,
   }
   // tcgen05 (tensor-memory accumulators) unless the warp-MMA kernel is asked
   // for, or the coarse keys need more shared memory than a CTA has
-  memset(&f.maps[3], 0, 2 * sizeof(CUtensorMap));
-  f.path = FwdPath::kMma;
-  if ((desc->flags & LLSA_FLAG_FWD_MMA_SYNC) == 0 && attn_fwd_tc_smem(f.p) <= kMaxSmemPerCta) {
-    f.path = FwdPath::kTc;
-    int st = make_row_tile_map(&f.maps[3], o, rows, desc->D, 128);
-    if (st == LLSA_OK && o_res != nullptr) st = make_row_tile_map(&f.maps[4], o_res, rows, desc->D, 128);
-    if (st != LLSA_OK) return st;
-  }
+  const bool tc_fits = attn_fwd_tc_smem(f.p) <= kMaxSmemPerCta;
+  f.path = ((desc->flags & LLSA_FLAG_FWD_MMA_SYNC) == 0 && tc_fits) ? FwdPath::kTc : FwdPath::kMma;
   f.p.o_res = o_res;
   return LLSA_OK;
 }

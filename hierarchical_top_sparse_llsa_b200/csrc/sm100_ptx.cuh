@@ -32,16 +32,20 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
+// One poll of phase `parity`; the thread may be suspended (issuing nothing)
+// for up to kPollSuspendNs while the phase is incomplete, and resumes as soon
+// as it completes.
+constexpr uint32_t kPollSuspendNs = 20000;
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n"
       ".reg .pred p;\n"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
       "selp.u32 %0, 1, 0, p;\n"
       "}\n"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(kPollSuspendNs)
       : "memory");
   return ok != 0;
 }
@@ -54,8 +58,8 @@ __device__ __forceinline__ uint64_t global_ns() {
 }
 
 // Wait for phase `parity` of a barrier for at most `limit_ns` nanoseconds of
-// the global timer (checked every 32 polls; a poll may itself suspend for a
-// short hardware-defined time).  Returns false on time-out; the caller then
+// the global timer (checked every 32 polls; a poll may itself suspend for up
+// to kPollSuspendNs, so the limit is overshot by at most about 1 ms).  Returns false on time-out; the caller then
 // reports LLSA_DEV_TIMEOUT.  The default limit, 1 s, is far above any wait of
 // a correct launch (the longest kernel of the path runs for about a
 // millisecond) and short enough that a lost arrival ends the launch instead

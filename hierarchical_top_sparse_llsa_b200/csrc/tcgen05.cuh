@@ -123,6 +123,24 @@ __device__ __forceinline__ void tmem_st32u(uint32_t taddr, const uint32_t (&v)[3
       : "memory");
 }
 
+// registers -> TMEM: 16 packed 32-bit words of this lane
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
+// registers -> TMEM: N (16 or 32) packed 32-bit words of this lane
+template <int N>
+__device__ __forceinline__ void tmem_st_words(uint32_t taddr, const uint32_t* v) {
+  static_assert(N == 16 || N == 32, "16 or 32 words");
+  if constexpr (N == 16) tmem_st16u(taddr, v);
+  else tmem_st32u(taddr, *reinterpret_cast<const uint32_t(*)[32]>(v));
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
