@@ -480,6 +480,7 @@ def run_ours(args, rank, world, local_rank):
     del x
     desc = llsa.make_desc(w.B, w.H, w.N, w.D, w.L, w.topk, llsa.BF16 if w.dtype == "bf16" else llsa.F32,
                           flags=(llsa.FLAG_FWD_MMA_SYNC if args.fwd_mma_sync else 0)
+                          | (llsa.FLAG_FWD_TCGEN05 if args.fwd_tcgen05 else 0)
                           | (llsa.FLAG_BWD_TCGEN05 if args.bwd_tcgen05 else 0))
     bufs = llsa.LlsaBuffers(desc, dev, with_bwd=w.backward)
     o = torch.empty_like(t_in["q"])
@@ -718,7 +719,8 @@ def run_ours(args, rank, world, local_rank):
     attn_flops = work["fwd"]["flops"] + (work["bwd"]["flops"] if w.backward else 0)
     sel_ms = stage_ms["pool"] + stage_ms["select"]
     # the fused call saves the level-1 selection launch on the bf16 warp-MMA forward
-    fused_saves = fuse and w.dtype == "bf16" and args.fwd_mma_sync
+    fwd_is_mma = args.fwd_mma_sync or (w.D == 64 and not args.fwd_tcgen05)
+    fused_saves = fuse and w.dtype == "bf16" and fwd_is_mma
     nlaunch = sum(launches_per_step(w.L)[n] for n in names) - (1 if fused_saves else 0)
     line = {
         "metric": METRIC, "value": world * tokens / (ms * 1e-3), "unit": UNIT, "n_gpus": world,
@@ -766,7 +768,9 @@ def main():
     ap.add_argument("--bwd-tcgen05", action="store_true",
                     help="run the key-major backward pass on the tcgen05 kernel (bf16, D=64)")
     ap.add_argument("--fwd-mma-sync", action="store_true",
-                    help="run the forward on the warp-level mma.sync kernel instead of the tcgen05 one (bf16)")
+                    help="force the forward onto the warp-level mma.sync kernel (bf16; the D=64 default)")
+    ap.add_argument("--fwd-tcgen05", action="store_true",
+                    help="force the forward onto the tcgen05 kernel (bf16; the D=128 default)")
     ap.add_argument("--no-transpose-graph", action="store_true",
                     help="skip the index transpose timed as back-to-back calls in a CUDA graph")
     ap.add_argument("--no-residual", action="store_true",

@@ -251,10 +251,16 @@ int plan_fwd(const llsa_desc* desc, const void* q, const void* k, const void* v,
     const int st = make_row_tile_map(&f.maps[i], srcs[i], rows, desc->D);
     if (st != LLSA_OK) return st;
   }
-  // tcgen05 (tensor-memory accumulators) unless the warp-MMA kernel is asked
-  // for, or the coarse keys need more shared memory than a CTA has
+  // Default: the faster of the two bf16 forwards as measured on B200 at the
+  // synthetic workloads -- tcgen05 at D = 128 (1.30 vs 2.24 ms at 512x512
+  // pixels, K = 8), the warp-MMA kernel at D = 64 (0.31 vs 0.55 ms at 256x256
+  // pixels).  The flags force either; tcgen05 also needs its coarse keys to
+  // fit in a CTA's shared memory.
   const bool tc_fits = attn_fwd_tc_smem(f.p) <= kMaxSmemPerCta;
-  f.path = ((desc->flags & LLSA_FLAG_FWD_MMA_SYNC) == 0 && tc_fits) ? FwdPath::kTc : FwdPath::kMma;
+  bool tc = desc->D == 128;
+  if (desc->flags & LLSA_FLAG_FWD_TCGEN05) tc = true;
+  if (desc->flags & LLSA_FLAG_FWD_MMA_SYNC) tc = false;
+  f.path = (tc && tc_fits) ? FwdPath::kTc : FwdPath::kMma;
   f.p.o_res = o_res;
   return LLSA_OK;
 }

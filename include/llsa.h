@@ -65,21 +65,24 @@ enum {
 
 /* descriptor flags */
 enum {
-  /* bf16: the forward on the tcgen05 kernel (tensor-memory accumulators, 8
-   * sibling query blocks per 128-row MMA).  This is the default for bf16; the
-   * flag states it explicitly and excludes LLSA_FLAG_FWD_MMA_SYNC. */
+  /* bf16: run the forward (llsa_attn_fwd, llsa_attn_fwd_res, the forward of
+   * llsa_select_attn_fwd) on the tcgen05 kernel: a persistent kernel whose
+   * groups of 8 sibling query blocks (128 rows, one MMA) walk the union of
+   * their selected key blocks with S and O in tensor memory.  Without a
+   * forward flag the library picks the faster kernel for the head dim, as
+   * measured on B200: tcgen05 at D = 128, the warp-MMA kernel at D = 64.
+   * Excludes LLSA_FLAG_FWD_MMA_SYNC. */
   LLSA_FLAG_FWD_TCGEN05 = 1,
   /* bf16, D = 64: run the key-major pass of llsa_attn_bwd (dK, dV) on the
    * tcgen05 kernel (8 query blocks of a key block per 128-row MMA, dK and dV
    * accumulated in tensor memory) instead of the warp-MMA kernel. */
   LLSA_FLAG_BWD_TCGEN05 = 2,
-  /* bf16: run the forward (llsa_attn_fwd, llsa_attn_fwd_res and the forward of
-   * llsa_select_attn_fwd) on the warp-level mma.sync kernel (one warp per 4
-   * query blocks, registers as accumulators) instead of the tcgen05 kernel,
-   * for comparison.  Both compute the same result within bf16 rounding.  The
-   * library also takes this kernel by itself when the coarse keys of one CTA
-   * need more shared memory than the tcgen05 kernel has (the sum of K_l over
-   * levels 2..Lc above 128 at D = 128). */
+  /* bf16: run the forward on the warp-level mma.sync kernel (one warp per 4
+   * query blocks, registers as accumulators, each block against exactly its
+   * own key blocks).  Both kernels compute the same result within bf16
+   * rounding.  The library also takes this kernel when the coarse keys of one
+   * CTA need more shared memory than the tcgen05 kernel has (the sum of K_l
+   * over levels 2..Lc above 128 at D = 128). */
   LLSA_FLAG_FWD_MMA_SYNC = 4
 };
 
@@ -197,8 +200,8 @@ LLSA_API int llsa_attn_fwd(const llsa_desc* desc, const void* q, const void* k, 
  *   and k[l], v[l] for l = 2..Lc; idx: I(1..L), all written (as llsa_select
  *   writes them; the backward needs them).  Results are identical to the two
  *   calls made one after the other.  The fusion is done by the warp-MMA
- *   forward (LLSA_FLAG_FWD_MMA_SYNC); on the tcgen05 forward (the bf16
- *   default) and in fp32 the level-1 selection runs as its own launch before
+ *   forward (the D = 64 default, or LLSA_FLAG_FWD_MMA_SYNC); with the tcgen05
+ *   forward and in fp32 the level-1 selection runs as its own launch before
  *   the forward.
  */
 LLSA_API int llsa_select_attn_fwd(const llsa_desc* desc, const void* q, const void* k, const void* v,

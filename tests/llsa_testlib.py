@@ -141,6 +141,63 @@ def run_oracle(inputs, L, topk, level_w=None, idx=None, bwd=True, pyr=None, enri
     return res
 
 
+# ---------------------------------------------------------------- near ties
+# North star's acceptance rule for selected indices: bit-exact, except that a
+# near tie may go either way.  The reading taken (the near-tie adjudication of
+# the build's reading list): compare level by level against the oracle's
+# selection *given the GPU's parent row* (so one tie does not cascade), and
+# accept a differing slot only if its fp32 score lies within the rounding
+# bound of the K-th kept score.  A dot product of length D summed in any order
+# in fp32 is within gamma_D * sum_d |q_d k_d| of the exact value,
+# gamma_D = D u / (1 - D u), u = 2^-24 (Higham, recursive summation); two
+# computed scores can cross when their exact values are within the sum of
+# their two bounds.  Outputs are then compared on the oracle's indices.
+
+def _gamma(D):
+    u = 2.0 ** -24
+    return D * u / (1.0 - D * u)
+
+
+def adjudicate_selection(pq, pk, gpu_idx, L, topk):
+    """Check the GPU's I(1..L) against the oracle level by level, conditional
+    on the GPU's parents.  Returns the number of rows that differ only by near
+    ties; raises AssertionError on any other difference.  pq, pk: the pooled
+    queries and keys (the GPU's equal the oracle's bit for bit); topk: K or a
+    {level: K_l} mapping."""
+    from oracle.llsa_oracle import _scores_fp32, candidates_for_level
+
+    kl = (lambda l: topk[l]) if isinstance(topk, dict) else (lambda l: topk)
+    near = 0
+    for l in range(L, 0, -1):
+        parent = None if l == L else np.asarray(gpu_idx[l + 1])
+        ref = oracle.select_level(pq[l], pk[l], parent, kl(l))
+        got = np.asarray(gpu_idx[l])
+        diff = np.argwhere((ref != got).any(-1))
+        for b, h, q in diff:
+            if parent is None:
+                cand = np.arange(pq[l].shape[2])
+            else:
+                cand = candidates_for_level(parent[b:b + 1, h:h + 1], 16)[0, 0, q // 16]
+                cand = cand[cand >= 0]
+            qv = np.asarray(pq[l][b, h, q], dtype=np.float32)
+            kv = np.asarray(pk[l][b, h][cand], dtype=np.float32)
+            s = _scores_fp32(qv[None], kv[None])[0].astype(np.float64)
+            bound = _gamma(qv.shape[-1]) * np.abs(qv.astype(np.float64)[None] * kv.astype(np.float64)).sum(-1)
+            pos = {int(c): i for i, c in enumerate(cand)}
+            kept_ref = [int(c) for c in ref[b, h, q] if c >= 0]
+            kept_got = [int(c) for c in got[b, h, q] if c >= 0]
+            assert len(kept_ref) == len(kept_got), (l, b, h, q, kept_ref, kept_got)
+            kth = min(kept_ref, key=lambda c: (s[pos[c]], -c))  # the oracle's last kept key
+            for c in set(kept_ref) ^ set(kept_got):
+                assert c in pos, (l, b, h, q, c, "not a candidate")
+                gap = abs(s[pos[c]] - s[pos[kth]])
+                assert gap <= bound[pos[c]] + bound[pos[kth]], (
+                    f"level {l} row {(int(b), int(h), int(q))}: key {c} differs by {gap:.3g}, "
+                    f"beyond the rounding bound {bound[pos[c]] + bound[pos[kth]]:.3g}")
+            near += 1
+    return near
+
+
 def workload_inputs(name, heads=None):
     w = workloads.WORKLOADS[name]
     return w, workloads.make_inputs(w, heads=heads, with_dout=w.backward)
