@@ -390,21 +390,49 @@ def gpu_selector(torch, dev):
 
 
 # ------------------------------------------------------------- CPU oracle
-def oracle_sample(w, x_head):
-    """The oracle's whole path on one head (a bounded sample of the workload)."""
+def oracle_sample(w, x_head, stages=None):
+    """The oracle's whole path on a head slice (a bounded sample of the
+    workload); returns the seconds it took and, in ``stages`` if given, the
+    seconds of each stage."""
     import oracle
 
     L, K = w.L, w.topk
     scale = oracle.default_scale(w.D)
+    st = {} if stages is None else stages
     t0 = time.perf_counter()
     pq, pk, pv = oracle.pool(x_head["q"], L), oracle.pool(x_head["k"], L), oracle.pool(x_head["v"], L)
+    t1 = time.perf_counter()
     idx = oracle.select_all(pq, pk, L, K)
+    t2 = time.perf_counter()
     O, LSE = oracle.attn_fwd(x_head["q"], x_head["k"], x_head["v"], pk, pv, idx, L, scale)
+    t3 = time.perf_counter()
+    st.update(pool=t1 - t0, select=t2 - t1, fwd=t3 - t2)
     if w.backward:
         for l in range(1, L + 1):
             oracle.index_transpose(idx[l], w.n_level(l))
+        t4 = time.perf_counter()
         oracle.attn_bwd(x_head["q"], x_head["k"], x_head["v"], pk, pv, O, LSE, x_head["do"], idx, L, scale)
+        t5 = time.perf_counter()
+        st.update(transpose=t4 - t3, bwd=t5 - t4)
     return time.perf_counter() - t0
+
+
+def oracle_one_thread(name="img64_bf16"):
+    """The oracle on one head of a small workload with one BLAS thread: the
+    single-core figure of the CPU baseline (seconds and tokens/s)."""
+    w = workloads.WORKLOADS[name]
+    x = workloads.make_inputs(w, heads=[0], with_dout=w.backward)
+    try:
+        from threadpoolctl import threadpool_limits
+    except Exception:  # threadpoolctl missing: report the default threads
+        threadpool_limits = None
+    if threadpool_limits is not None:
+        with threadpool_limits(limits=1):
+            t = oracle_sample(w, x)
+    else:
+        t = oracle_sample(w, x)
+    return {"workload": name, "sample": "head 0 (B*N/H tokens)", "threads": 1 if threadpool_limits else None,
+            "seconds": round(t, 3), "tokens/s": round(w.B * w.N / w.H / t, 1)}
 
 
 def blas_threads():
@@ -422,11 +450,18 @@ def cpu_sample_inputs(w):
     return x
 
 
+L2_BYTES = 126 * 2**20  # B200
+
+
 def config_of(w, world):
+    es = 2 if w.dtype == "bf16" else 4
+    inputs = (4 if w.backward else 3) * w.B * w.H * w.N * w.D * es
+    l2 = ("inputs larger than L2 (no flush needed)" if inputs > L2_BYTES else
+          f"inputs {inputs / 2**20:.1f} MiB fit in L2: warm-cache timing (a small parity workload)")
     return {"workload": f"{w.name}: {w.side}x{w.side} pixels, N={w.N}, B={w.B}, H={w.H}, D={w.D}, "
                         f"L={w.L}, K={w.topk}, {'fwd+bwd' if w.backward else 'fwd only'}",
             "B": w.B, "H": w.H, "N": w.N, "D": w.D, "L": w.L, "topk": w.topk,
-            "l2": "inputs larger than L2 (no flush needed)",
+            "l2": l2,
             "parallelism": f"replicas x{world} (no collective)"}
 
 
@@ -469,9 +504,12 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         nh = min(4, w.H)
         xc = workloads.make_inputs(w, heads=slice(0, nh), with_dout=w.backward)
-        t = oracle_sample(w, xc)
+        stage_s = {}
+        t = oracle_sample(w, xc, stage_s)
         cpu = {"value": w.B * w.N * nh / w.H / t, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-               "sample": f"oracle whole path on heads 0..{nh - 1} of {w.H} ({t:.1f} s)"}
+               "sample": f"oracle whole path on heads 0..{nh - 1} of {w.H} ({t:.1f} s)",
+               "stage_seconds": {k: round(v, 3) for k, v in stage_s.items()},
+               "one_thread": oracle_one_thread()}
 
     x = workloads.make_inputs(w, with_dout=w.backward)
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
