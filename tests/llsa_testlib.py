@@ -198,6 +198,23 @@ def adjudicate_selection(pq, pk, gpu_idx, L, topk):
     return near
 
 
+def settle_indices(g, r, x, L, topk, dtype, sl=(slice(None), slice(None)), bwd=True, **run_kw):
+    """Indices of the GPU run ``g`` against the oracle's ``r``: equal, or
+    differing by near ties only (adjudicated), in which case the path is run
+    again on the GPU over the oracle's indices for the heads of ``x``.
+    Returns (the run whose outputs to compare, its head slice, the number of
+    adjudicated rows)."""
+    gidx = {l: g["idx"][l][sl] for l in range(1, L + 1)}
+    if all(np.array_equal(gidx[l], r["idx"][l]) for l in gidx):
+        return g, sl, 0
+    near = adjudicate_selection(r["pq"], r["pk"], gidx, L, topk)
+    print(f"{near} index rows differ by near ties only (adjudicated)")
+    B, H, N, D = x["q"].shape
+    g2 = run_gpu(B, H, N, D, L, topk if not isinstance(topk, dict) else max(topk.values()), dtype, x,
+                 ext_idx=r["idx"], bwd=bwd, **run_kw)
+    return g2, (slice(None), slice(None)), near
+
+
 def workload_inputs(name, heads=None):
     w = workloads.WORKLOADS[name]
     return w, workloads.make_inputs(w, heads=heads, with_dout=w.backward)

@@ -7,7 +7,7 @@ import pytest
 
 import hierarchical_top_sparse_llsa_b200 as llsa
 from hierarchical_top_sparse_llsa_b200 import workloads
-from llsa_testlib import assert_close, run_gpu, run_oracle
+from llsa_testlib import assert_close, run_gpu, run_oracle, settle_indices
 
 pytestmark = pytest.mark.gpu
 
@@ -18,10 +18,9 @@ def _small(seed, B, H, N, D, dtype="bf16"):
     return {k: workloads.round_to_bf16(v) for k, v in x.items()} if dtype == "bf16" else x
 
 
-def _check(g, r, L, dtype, hs=slice(None)):
+def _check(g, r, L, dtype, hs=slice(None), x=None, topk=8, **run_kw):
     sl = (slice(None), hs)  # heads are axis 1
-    for l in range(1, L + 1):
-        assert np.array_equal(g["idx"][l][sl], r["idx"][l]), f"indices level {l}"
+    g, sl, _ = settle_indices(g, r, x, L, topk, dtype, sl, resid=True, **run_kw)
     assert_close(g["O"][sl], r["O"], dtype, "O")
     assert_close(g["LSE"][sl], r["LSE"], "f32" if dtype == "f32" else "bf16", "LSE")
     for name in ("dQ", "dK", "dV"):
@@ -41,7 +40,7 @@ def test_workloads(name, heads):
     hs = slice(None) if heads is None else heads
     xs = x if heads is None else {k: np.ascontiguousarray(v[:, heads]) for k, v in x.items()}
     r = run_oracle(xs, w.L, w.topk)
-    _check(g, r, w.L, w.dtype, hs)
+    _check(g, r, w.L, w.dtype, hs, x=xs)
 
 
 @pytest.mark.parametrize("B,H,N,D,L,kw", [
@@ -58,7 +57,7 @@ def test_variants(B, H, N, D, L, kw):
     assert g["status"] == 0
     topk = 8 if "topk_l" not in kw else {l: kw["topk_l"][l] or 8 for l in range(1, L + 1)}
     r = run_oracle(x, L, topk, level_w=kw.get("level_w"), enrich=kw.get("enrich") or None)
-    _check(g, r, L, "bf16")
+    _check(g, r, L, "bf16", x=x, topk=topk, **kw)
 
 
 def test_forward_outputs_and_residual_bound():
@@ -73,7 +72,7 @@ def test_forward_outputs_and_residual_bound():
     assert np.all(np.isfinite(R))
     half_ulp = np.ldexp(1.0, np.frexp(np.abs(O))[1] - 9)  # half a bf16 step at |O|
     assert np.all(np.abs(R) <= half_ulp * (1 + 2.0**-7) + 1e-30)
-    r = run_oracle(x, L, 8, bwd=False)
+    r = run_oracle(x, L, 8, bwd=False, idx=g["idx"])  # attention on the GPU's own indices
     err_plain = np.sqrt(np.mean((O - r["O"]) ** 2))
     err_res = np.sqrt(np.mean((O + R - r["O"]) ** 2))
     assert err_res < err_plain
