@@ -34,6 +34,7 @@ NOALLOC_SCRATCH_BYTES = 16 << 20
 
 EXPORTED = (
     "llsa_pool",
+    "llsa_qkv_pool",
     "llsa_select",
     "llsa_attn_fwd",
     "llsa_select_attn_fwd",
@@ -99,6 +100,7 @@ def lib() -> ctypes.CDLL:
         vp, P = ctypes.c_void_p, ctypes.POINTER
         sig = {
             "llsa_pool": (ctypes.c_int, [P(LlsaDesc), vp, vp, vp, P(LlsaPyramid), vp]),
+            "llsa_qkv_pool": (ctypes.c_int, [P(LlsaDesc), vp, vp, ctypes.c_int, vp, vp, vp, P(LlsaPyramid), vp, vp]),
             "llsa_select": (ctypes.c_int, [P(LlsaDesc), P(LlsaPyramid), P(LlsaIndices), vp]),
             "llsa_attn_fwd": (ctypes.c_int, [P(LlsaDesc), vp, vp, vp, P(LlsaPyramid), P(LlsaIndices),
                                              vp, vp, vp, vp]),
@@ -176,6 +178,11 @@ def level_topk(desc: LlsaDesc, l: int) -> int:
 # ------------------------------------------------------------ entry points
 def llsa_pool(desc, q, k, v, pyramid, stream=0, check=True):
     st = lib().llsa_pool(ctypes.byref(desc), q, k, v, ctypes.byref(pyramid), stream)
+    return _check(st) if check else st
+
+
+def llsa_qkv_pool(desc, x, w, C, q, k, v, pyramid, dev_status=None, stream=0, check=True):
+    st = lib().llsa_qkv_pool(ctypes.byref(desc), x, w, C, q, k, v, ctypes.byref(pyramid), dev_status, stream)
     return _check(st) if check else st
 
 

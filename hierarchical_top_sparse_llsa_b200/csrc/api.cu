@@ -18,6 +18,8 @@ cudaError_t launch_attn_fwd_mma_select(const AttnParams& p, const SelectParams& 
 cudaError_t launch_attn_fwd_tc(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s);
 size_t attn_fwd_tc_smem(const AttnParams& p);
 cudaError_t launch_attn_bwd_mma(const AttnParams& p, const CUtensorMap* maps, cudaStream_t s, bool tc_kv);
+cudaError_t launch_qkv_pool(const CUtensorMap* maps, void* const out[3], float* const lvl[3][3], int32_t* status,
+                            int B, int N, int H, int D, int L, int C, cudaStream_t s);
 }  // namespace llsa
 
 using namespace llsa;
@@ -147,6 +149,23 @@ int make_row_tile_map(CUtensorMap* map, const void* base, uint64_t rows, int D) 
   const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
   const cuuint32_t box[2] = {64, 16};
+  const cuuint32_t estride[2] = {1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? LLSA_OK : LLSA_ERR_LAUNCH;
+}
+
+// A bf16 [rows, cols] row-major matrix seen by TMA as boxes of box_rows rows
+// x 64 columns (128 bytes) with 128-byte swizzle.
+int make_kslice_map(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_tiled();
+  if (fn == nullptr) return LLSA_ERR_LAUNCH;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) != 0) return LLSA_ERR_INVALID_ARG;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {64, box_rows};
   const cuuint32_t estride[2] = {1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                         strides, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -337,6 +356,53 @@ int llsa_pool(const llsa_desc* desc, const void* q, const void* k, const void* v
   p.D = desc->D;
   p.L = desc->L;
   return launch_status(launch_pool(p, desc->dtype, (cudaStream_t)stream));
+}
+
+int llsa_qkv_pool(const llsa_desc* desc, const void* x, const void* w, int C, void* q, void* k, void* v,
+                  const llsa_pyramid* out, int32_t* dev_status, void* stream) {
+  int st = check_desc(desc);
+  if (st != LLSA_OK) return st;
+  if (x == nullptr || w == nullptr || q == nullptr || k == nullptr || v == nullptr || out == nullptr)
+    return LLSA_ERR_INVALID_ARG;
+  if (C < 64 || C % 64 != 0) return LLSA_ERR_INVALID_ARG;
+  if (desc->dtype != LLSA_BF16 || (desc->H * desc->D) % 128 != 0 || desc->N % 256 != 0)
+    return LLSA_ERR_UNSUPPORTED;
+  const void* ptrs[5] = {x, w, q, k, v};
+  for (const void* ptr : ptrs)
+    if ((reinterpret_cast<uintptr_t>(ptr) & 15) != 0) return LLSA_ERR_INVALID_ARG;
+  for (int l = 1; l <= desc->L; ++l) {
+    if (out->q[l] == nullptr || out->k[l] == nullptr) return LLSA_ERR_INVALID_ARG;
+    if (l >= 2 && out->v[l] == nullptr) return LLSA_ERR_INVALID_ARG;
+  }
+  const long long tokens = (long long)desc->B * desc->N;
+  const int HD = desc->H * desc->D;
+  CUtensorMap maps[2];
+  st = make_kslice_map(&maps[0], x, (uint64_t)tokens, (uint64_t)C, 256);
+  if (st != LLSA_OK) return st;
+  st = make_kslice_map(&maps[1], w, (uint64_t)3 * HD, (uint64_t)C, 128);
+  if (st != LLSA_OK) return st;
+  void* const o[3] = {q, k, v};
+  float* const lvl[3][3] = {{nullptr, out->q[1], desc->L >= 2 ? out->q[2] : nullptr},
+                            {nullptr, out->k[1], desc->L >= 2 ? out->k[2] : nullptr},
+                            {nullptr, nullptr, desc->L >= 2 ? out->v[2] : nullptr}};
+  cudaError_t e = launch_qkv_pool(maps, o, lvl, dev_status, desc->B, desc->N, desc->H, desc->D, desc->L, C,
+                                  (cudaStream_t)stream);
+  if (e != cudaSuccess) return LLSA_ERR_LAUNCH;
+  if (desc->L >= 3) {
+    PoolParams p;
+    memset(&p, 0, sizeof(p));
+    for (int l = 1; l <= desc->L; ++l) {
+      p.lvl[0][l] = out->q[l];
+      p.lvl[1][l] = out->k[l];
+      p.lvl[2][l] = (l >= 2) ? out->v[l] : nullptr;
+    }
+    p.BH = desc->B * desc->H;
+    p.N = desc->N;
+    p.D = desc->D;
+    p.L = desc->L;
+    e = launch_pool_up(p, (cudaStream_t)stream);
+  }
+  return launch_status(e);
 }
 
 int llsa_select(const llsa_desc* desc, const llsa_pyramid* pyr, const llsa_indices* out,

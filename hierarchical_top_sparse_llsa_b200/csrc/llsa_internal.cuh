@@ -184,6 +184,7 @@ struct AttnParams {
 // ------------------------------------------------------ kernel launchers
 // Each returns cudaSuccess or the launch error.
 cudaError_t launch_pool(const PoolParams& p, int dtype, cudaStream_t s);
+cudaError_t launch_pool_up(const PoolParams& p, cudaStream_t s);  // levels 3..L from level 2
 cudaError_t launch_select_level(const SelectParams& p, int BH, int D, cudaStream_t s);
 cudaError_t launch_transpose(const TransposeParams& p, cudaStream_t s);
 void transpose_chunking(int n, int* nchunk, int* rows);

@@ -108,6 +108,11 @@ cudaError_t launch_pool(const PoolParams& p, int dtype, cudaStream_t s) {
   else
     e = (p.D == 64) ? launch_l12<float, 64>(p, s) : launch_l12<float, 128>(p, s);
   if (e != cudaSuccess) return e;
+  return launch_pool_up(p, s);
+}
+
+cudaError_t launch_pool_up(const PoolParams& p, cudaStream_t s) {
+  cudaError_t e;
   for (int l = 3; l <= p.L; ++l) {
     const size_t total = (size_t)p.BH * (p.N >> (4 * l)) * p.D;
     int blocks = (int)((total + 255) / 256);

@@ -154,6 +154,26 @@ LLSA_API int llsa_pool(const llsa_desc* desc, const void* q, const void* k, cons
               const llsa_pyramid* out, void* stream);
 
 /*
+ * llsa_qkv_pool - the QKV projection with the hierarchical compression in
+ * its epilogue: the step before the path ("Input (Q, K, V) -> Hierarchical
+ * Compression -> ..." in the pipeline overview; Step 1, Building Blocks:
+ * Hierarchical Compression), fused so that Q, K and V are not read back.
+ *   [Q | K | V] = X W^T on the tensor cores (bf16 inputs, fp32 accumulation,
+ *   each output rounded once to bf16).  x: bf16 [B, N, C] row-major, tokens
+ *   in Z-order; w: bf16 [3*H*D, C] row-major (a linear layer's weight: output
+ *   feature t*H*D + h*D + d is tensor t = 0 Q, 1 K, 2 V, head h, channel d).
+ *   q, k, v: written, bf16 [B, H, N, D] as the other calls take them.  out:
+ *   the pyramid, written exactly as llsa_pool would write it from these q, k,
+ *   v (bit for bit); every level listed in llsa_pyramid is required.
+ *   Requires dtype LLSA_BF16, H*D a multiple of 128 and N a multiple of 256
+ *   (else LLSA_ERR_UNSUPPORTED); C a positive multiple of 64 and every
+ *   pointer 16-byte aligned (else LLSA_ERR_INVALID_ARG).  dev_status (may be
+ *   NULL): LLSA_DEV_TIMEOUT if a bounded wait of the kernel gave up.
+ */
+LLSA_API int llsa_qkv_pool(const llsa_desc* desc, const void* x, const void* w, int C, void* q, void* k,
+                           void* v, const llsa_pyramid* out, int32_t* dev_status, void* stream);
+
+/*
  * llsa_select - hierarchical Top-K selection (Step 2; Building Blocks:
  * Hierarchical Top-K Selection).
  *   Level L: every level-L query token scores every level-L key token.
