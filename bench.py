@@ -172,6 +172,74 @@ def dense_reference(torch, w, dev, iters=3):
             "fwd_ms": round(fwd_ms, 3), "fwd_bwd_ms": round(fb_ms, 3), "iters": iters}
 
 
+def qkv_projection(torch, llsa, w, dev, pool_ms, step_ms, tens, iters=10):
+    """The step before the path: the QKV projection of a model of width
+    C = H * D, fused with the pool (llsa_qkv_pool: tcgen05 GEMM whose epilogue
+    writes Q, K, V head-major and the pyramid) against the unfused sequence
+    (cuBLAS GEMM through torch.matmul, the head-major relayout, llsa_pool).
+    Reports both and the step time with each in front of it.  Not part of the
+    timed step."""
+    C = w.H * w.D
+    if w.dtype != "bf16" or C % 128 != 0 or w.N % 256 != 0:
+        return None
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(777)
+    x = torch.randn(w.B, w.N, C, device=dev, dtype=torch.bfloat16, generator=gen)
+    wt = (torch.randn(3 * C, C, device=dev, generator=gen) / C ** 0.5).to(torch.bfloat16)
+    desc = llsa.make_desc(w.B, w.H, w.N, w.D, w.L, w.topk, llsa.BF16)
+    fused = llsa.LlsaBuffers(desc, dev, with_bwd=False)
+    plain = llsa.LlsaBuffers(desc, dev, with_bwd=False)
+    qkv = [torch.empty(w.B, w.H, w.N, w.D, device=dev, dtype=torch.bfloat16) for _ in range(3)]
+    sh = torch.cuda.current_stream(dev).cuda_stream
+    holder = {}
+
+    def fused_call():
+        llsa.llsa_qkv_pool(desc, x.data_ptr(), wt.data_ptr(), C, qkv[0].data_ptr(), qkv[1].data_ptr(),
+                           qkv[2].data_ptr(), fused.pyramid, fused.status.data_ptr(), sh)
+
+    def gemm():
+        holder["y"] = torch.matmul(x.view(-1, C), wt.t())
+
+    def relayout():
+        holder["t"] = holder["y"].view(w.B, w.N, 3, w.H, w.D).permute(2, 0, 3, 1, 4).contiguous()
+
+    def pool():
+        t = holder["t"]
+        llsa.llsa_pool(desc, t[0].data_ptr(), t[1].data_ptr(), t[2].data_ptr(), plain.pyramid, sh)
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(iters):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / iters
+
+    f_ms = timed(fused_call)
+    g_ms = timed(gemm)
+    r_ms = timed(relayout)
+    p_ms = timed(pool)
+    if int(fused.status.item()) != 0:
+        raise RuntimeError(f"llsa_qkv_pool device status {int(fused.status.item())}")
+    flops = 2.0 * w.B * w.N * C * 3 * C
+    unfused = g_ms + r_ms + p_ms
+    out = {"C": C, "flops": flops, "iters": iters, "l2": "X larger than L2" if x.numel() * 2 > L2_BYTES else "X in L2",
+           "fused_ms": round(f_ms, 4), "fused_TFLOPs": round(flops / (f_ms * 1e-3) / 1e12, 1),
+           "fused_frac_bf16_tensor": round(flops / (f_ms * 1e-3) / 1e12 / tens, 4),
+           "cublas_gemm_ms": round(g_ms, 4), "cublas_TFLOPs": round(flops / (g_ms * 1e-3) / 1e12, 1),
+           "relayout_ms": round(r_ms, 4), "pool_ms": round(p_ms, 4), "unfused_ms": round(unfused, 4),
+           "step_ms_with_projection": {"fused": round(step_ms - pool_ms + f_ms, 4),
+                                       "unfused": round(step_ms - pool_ms + unfused, 4)}}
+    del x, wt, fused, plain, qkv, holder
+    torch.cuda.empty_cache()
+    return out
+
+
 def max_over_ranks(torch, dist, values, device) -> list:
     """Element-wise maximum of per-rank timings (one all_reduce): the job's
     time is its slowest rank's."""
@@ -742,6 +810,7 @@ def run_ours(args, rank, world, local_rank):
     roof["kernel"] = f"llsa_{'attn_' if dom in ('fwd', 'bwd') else ''}{dom} ({launches_per_step(w.L)[dom]} launches)"
     roof["peak_source"] = f"{peaks['source']} (MEASURED_PEAKS.json)" if peaks["source"] == "measured" else "fallback"
     reorder = reorder_rate(torch, llsa, w, dev, t_in["q"], peaks["hbm_gbs"])
+    proj = None if args.no_projection else qkv_projection(torch, llsa, w, dev, stage_ms["pool"], ms, tens)
     tr_graph = None
     if w.backward and not args.no_transpose_graph:
         tr_graph = {"headline": transpose_graph_rate(torch, llsa, desc, bufs, dev, hbm, work["transpose"]["bytes"])}
@@ -777,6 +846,7 @@ def run_ours(args, rank, world, local_rank):
         "cpu_baseline": cpu,
         "dense_reference": dense,
         "reorder": reorder,
+        "qkv_projection": proj,
         "e2e": {"value": world * tokens / (e2e_ms * 1e-3), "unit": UNIT, "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "pipelined": "uploads of step k+1 and downloads of step k-1 overlap step k"},
@@ -814,6 +884,8 @@ def main():
     ap.add_argument("--no-residual", action="store_true",
                     help="time llsa_attn_fwd + llsa_attn_bwd (two walks of each key list) instead of the "
                          "_res calls (Delta from the bf16 residual of O)")
+    ap.add_argument("--no-projection", action="store_true",
+                    help="skip the QKV-projection comparison (llsa_qkv_pool against cuBLAS + llsa_pool)")
     ap.add_argument("--fuse-select", action="store_true",
                     help="time llsa_select_attn_fwd (level-1 selection in the forward's prologue) "
                          "instead of llsa_select + llsa_attn_fwd")
