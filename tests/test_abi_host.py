@@ -248,3 +248,30 @@ def test_wait_timeout_selftest_checks_arguments(lib):
     assert llsa.llsa_selftest_wait_timeout(None, 10, check=False) == llsa.ERR_INVALID_ARG
     assert llsa.llsa_selftest_wait_timeout(256, 0, check=False) == llsa.ERR_INVALID_ARG
     assert llsa.llsa_selftest_wait_timeout(256, 2000001, check=False) == llsa.ERR_INVALID_ARG
+
+
+def test_qkv_pool_checks_arguments(lib):
+    # every check below comes before the tensor maps are encoded or anything
+    # is launched: nothing reaches a device here
+    def pyramid(L):
+        pyr = llsa.LlsaPyramid()
+        for l in range(1, L + 1):
+            pyr.q[l] = pyr.k[l] = 256
+            if l >= 2:
+                pyr.v[l] = 256
+        return pyr
+
+    def call(d, x=256, w=256, C=128, q=256, k=256, v=256, pyr=None):
+        return llsa.llsa_qkv_pool(d, x, w, C, q, k, v, pyramid(d.L) if pyr is None else pyr, None, 0,
+                                  check=False)
+
+    d = llsa.make_desc(1, 2, 4096, 64, 3, 8, llsa.BF16)
+    assert call(d, x=None) == llsa.ERR_INVALID_ARG
+    assert call(d, v=None) == llsa.ERR_INVALID_ARG
+    assert call(d, C=0) == llsa.ERR_INVALID_ARG
+    assert call(d, C=96) == llsa.ERR_INVALID_ARG            # not a multiple of 64
+    assert call(d, w=264) == llsa.ERR_INVALID_ARG           # not 16-byte aligned
+    assert call(d, pyr=llsa.LlsaPyramid()) == llsa.ERR_INVALID_ARG  # pyramid levels missing
+    assert call(llsa.make_desc(1, 2, 4096, 64, 3, 8, llsa.F32)) == llsa.ERR_UNSUPPORTED
+    assert call(llsa.make_desc(1, 3, 4096, 64, 3, 8, llsa.BF16)) == llsa.ERR_UNSUPPORTED  # H*D = 192
+    assert call(llsa.make_desc(1, 2, 16, 64, 1, 8, llsa.BF16)) == llsa.ERR_UNSUPPORTED    # N = 16 < 256
