@@ -822,6 +822,19 @@ def run_ours(args, rank, world, local_rank):
         dense["llsa_fwd_bwd_ms"] = round(stage_ms["fwd"] + stage_ms["bwd"], 4)
         dense["speedup_fwd"] = round(dense["fwd_ms"] / stage_ms["fwd"], 2)
         dense["speedup_fwd_bwd"] = round(dense["fwd_bwd_ms"] / dense["llsa_fwd_bwd_ms"], 2)
+        # (query, key) pairs per second through each: dense attention scores all
+        # N^2 pairs of a head, the sparse path B*H*N*keys-per-query; the
+        # kernels' own dense form (every block selected, L = 1) would need rows
+        # of N/16 keys, beyond the K <= 32 their selection rows hold
+        dense_pairs = w.B * w.H * float(w.N) ** 2
+        sparse_pairs = w.B * w.H * float(w.N) * w.keys_per_query()
+        dense["pairs_per_s"] = {
+            "dense_fwd": dense_pairs / (dense["fwd_ms"] * 1e-3),
+            "llsa_fwd": sparse_pairs / (stage_ms["fwd"] * 1e-3),
+            "dense_fwd_bwd": dense_pairs / (dense["fwd_bwd_ms"] * 1e-3),
+            "llsa_fwd_bwd": sparse_pairs / (dense["llsa_fwd_bwd_ms"] * 1e-3),
+            "keys_per_query": w.keys_per_query(),
+        }
     attn_ms = stage_ms["fwd"] + stage_ms.get("bwd", 0.0)
     attn_flops = work["fwd"]["flops"] + (work["bwd"]["flops"] if w.backward else 0)
     sel_ms = stage_ms["pool"] + stage_ms["select"]
